@@ -1,0 +1,476 @@
+/*
+ * kvq_oracle.c -- plain, slow, obviously-correct CPU oracle for the quantized
+ * KV-cache decode path (calibration abs-max, FP8/NVFP4/BF16 quantize-on-write
+ * into a paged cache, dequantisation, and float64 decode attention).
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product library calls, links or
+ * includes this file; only the tests, the smoke check and the benchmark's
+ * CPU-baseline leg load it.  It shares no source with the CUDA path: the two
+ * agree only on the documented data layout and the formulas below.
+ *
+ * Every step follows the definitions as written, in the order written, with no
+ * blocking, fusion or reordering.  Sources:
+ *   [FP8-KV] "FP8 KV calibration guide" (thetechpanda.github.io,
+ *            radiance-R9700-vllm-experiments), the paragraph on the Radiance
+ *            calibrator: per-layer abs-max of BF16 K/V activations, OCP E4M3
+ *            convention, scale = max(observed_absolute_max * 1.05 / 448, 1e-12);
+ *            and the paragraph on storage: BF16 uses 2 bytes per element, FP8 one.
+ *   [NVFP4]  "I Tested NVFP4 vs FP8 KV Cache on Blackwell (One Refused to Boot)",
+ *            "What you'll learn": E4M3 at one byte per number; NVFP4 is a
+ *            block-scaled 4-bit float with FP8 scale factors, 4.5 bits per
+ *            number.  The block recipe used here (16-element E2M1 blocks along
+ *            head_dim, E4M3 block scale = block_absmax / (6 g), FP32 per-tensor
+ *            g = tensor_absmax / (448 * 6)) is the recipe this library
+ *            implements; the page fixes only the format family and its size.
+ *   OCP 8-bit floating point specification (E4M3: bias 7, no infinities,
+ *            S.1111.111 is NaN, max finite 448) and the OCP MX specification
+ *            (E2M1: bias 1, magnitudes 0, .5, 1, 1.5, 2, 3, 4, 6, no NaN/Inf).
+ *
+ * Parity status: every function here is pinned by a test that checks it
+ * against something other than itself (library conversions, brute force,
+ * closed forms, the pages' byte counts); see the tests directory.
+ */
+#include <float.h>
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* Format ids used by this oracle's C interface. */
+#define ORC_BF16 0
+#define ORC_FP8 1
+#define ORC_NVFP4 2
+
+#define ORC_PAGE 16 /* tokens per cache page (block size) */
+
+/* ------------------------------------------------------------------------ */
+/* BF16                                                                     */
+/* ------------------------------------------------------------------------ */
+
+/* A BF16 value is the upper half of an IEEE binary32; widening is exact. */
+static float bf16_to_f32(uint16_t b) {
+  uint32_t u = (uint32_t)b << 16;
+  float f;
+  memcpy(&f, &u, 4);
+  return f;
+}
+
+float orc_bf16_to_f32(uint16_t b) { return bf16_to_f32(b); }
+
+/* ------------------------------------------------------------------------ */
+/* E4M3 (OCP FP8, "FN" flavour): 1 sign, 4 exponent bits (bias 7), 3 mantissa */
+/* ------------------------------------------------------------------------ */
+
+/* Decode from the bit fields.  exponent 0: (m/8) * 2^-6 (subnormal);
+ * otherwise (1 + m/8) * 2^(e-7); S.1111.111 is NaN; there are no infinities. */
+float orc_e4m3_decode(uint8_t c) {
+  int s = (c >> 7) & 1;
+  int e = (c >> 3) & 0xF;
+  int m = c & 7;
+  double v;
+  if (e == 15 && m == 7) return NAN;
+  if (e == 0)
+    v = ((double)m / 8.0) * ldexp(1.0, -6);
+  else
+    v = (1.0 + (double)m / 8.0) * ldexp(1.0, e - 7);
+  return (float)(s ? -v : v);
+}
+
+/* Round a non-negative double q to the nearest integer, ties to even. */
+static double round_half_even(double q) {
+  double f = floor(q);
+  double r = q - f;
+  if (r > 0.5) return f + 1.0;
+  if (r < 0.5) return f;
+  return (fmod(f, 2.0) == 0.0) ? f : f + 1.0;
+}
+
+/* Encode by arithmetic on the binade: round to nearest, ties to even,
+ * saturating to +-448 (satfinite); the sign is kept for results that round to
+ * zero.  NaN inputs are outside the contract (returns the NaN code). */
+uint8_t orc_e4m3_encode(float x) {
+  uint8_t sign = signbit(x) ? 0x80 : 0x00;
+  double a = fabs((double)x);
+  if (isnan(x)) return (uint8_t)(sign | 0x7F);
+  if (a >= 448.0) return (uint8_t)(sign | 0x7E);
+  if (a < ldexp(1.0, -6)) {
+    /* subnormal range: step 2^-9; a result of 8 steps is the smallest normal */
+    double q = round_half_even(a / ldexp(1.0, -9));
+    return (uint8_t)(sign | (uint8_t)q); /* q in 0..8; 8 == code 0x08 */
+  }
+  int e2;
+  frexp(a, &e2); /* a = f * 2^e2, f in [0.5, 1) -> binade exponent e2-1 */
+  int e = e2 - 1;
+  double q = round_half_even(a / ldexp(1.0, e - 3)); /* in [8, 16] */
+  if (q == 16.0) {
+    q = 8.0;
+    e += 1;
+  }
+  int code = ((e + 7) << 3) | ((int)q - 8);
+  if (code > 0x7E) code = 0x7E; /* cannot happen below 448; kept for clarity */
+  return (uint8_t)(sign | code);
+}
+
+/* Brute force: scan the finite codes of the input's sign in increasing value
+ * and keep the nearest one.  "Nearer" is decided against the exact midpoint of
+ * the two candidates (representable in double), so huge inputs do not tie on
+ * rounded distances; at a midpoint the code with mantissa LSB 0 wins.  Inputs
+ * beyond the largest finite value therefore land on +-448 (satfinite). */
+uint8_t orc_e4m3_encode_nearest(float x) {
+  uint8_t sign = signbit(x) ? 0x80 : 0x00;
+  double a = fabs((double)x);
+  int best = 0;
+  for (int c = 1; c <= 0x7E; c++) {
+    double mid = ((double)orc_e4m3_decode((uint8_t)best) + (double)orc_e4m3_decode((uint8_t)c)) / 2;
+    if (a > mid || (a == mid && (c & 1) == 0)) best = c;
+  }
+  return (uint8_t)(sign | best);
+}
+
+/* ------------------------------------------------------------------------ */
+/* E2M1 (OCP MX FP4): 1 sign (bit 3), 2 exponent bits (bias 1), 1 mantissa   */
+/* ------------------------------------------------------------------------ */
+
+float orc_e2m1_decode(uint8_t c) {
+  int s = (c >> 3) & 1;
+  int e = (c >> 1) & 3;
+  int m = c & 1;
+  double v = (e == 0) ? 0.5 * m : (1.0 + 0.5 * m) * ldexp(1.0, e - 1);
+  return (float)(s ? -v : v);
+}
+
+uint8_t orc_e2m1_encode(float x) {
+  uint8_t sign = signbit(x) ? 0x8 : 0x0;
+  double a = fabs((double)x);
+  if (isnan(x)) return (uint8_t)(sign | 0x7); /* outside the contract */
+  if (a >= 6.0) return (uint8_t)(sign | 0x7);
+  if (a < 1.0) {
+    double q = round_half_even(a / 0.5); /* 0, 1 or 2 (2 == code 2 == 1.0) */
+    return (uint8_t)(sign | (uint8_t)q);
+  }
+  int e2;
+  frexp(a, &e2);
+  int e = e2 - 1;                                     /* 0, 1 or 2 */
+  double q = round_half_even(a / ldexp(1.0, e - 1)); /* in [2, 4] */
+  if (q == 4.0) {
+    q = 2.0;
+    e += 1;
+  }
+  int code = ((e + 1) << 1) | ((int)q - 2);
+  if (code > 7) code = 7;
+  return (uint8_t)(sign | code);
+}
+
+/* Brute force over the 8 magnitudes, as for E4M3. */
+uint8_t orc_e2m1_encode_nearest(float x) {
+  uint8_t sign = signbit(x) ? 0x8 : 0x0;
+  double a = fabs((double)x);
+  int best = 0;
+  for (int c = 1; c <= 7; c++) {
+    double mid = ((double)orc_e2m1_decode((uint8_t)best) + (double)orc_e2m1_decode((uint8_t)c)) / 2;
+    if (a > mid || (a == mid && (c & 1) == 0)) best = c;
+  }
+  return (uint8_t)(sign | best);
+}
+
+/* Array forms for exhaustive sweeps.  which: 0 = arithmetic, 1 = brute force. */
+void orc_e4m3_encode_array(const float* x, uint8_t* out, int64_t n, int which) {
+  for (int64_t i = 0; i < n; i++)
+    out[i] = which ? orc_e4m3_encode_nearest(x[i]) : orc_e4m3_encode(x[i]);
+}
+void orc_e2m1_encode_array(const float* x, uint8_t* out, int64_t n, int which) {
+  for (int64_t i = 0; i < n; i++)
+    out[i] = which ? orc_e2m1_encode_nearest(x[i]) : orc_e2m1_encode(x[i]);
+}
+void orc_e4m3_decode_array(const uint8_t* c, float* out, int64_t n) {
+  for (int64_t i = 0; i < n; i++) out[i] = orc_e4m3_decode(c[i]);
+}
+void orc_e2m1_decode_array(const uint8_t* c, float* out, int64_t n) {
+  for (int64_t i = 0; i < n; i++) out[i] = orc_e2m1_decode(c[i] & 0xF);
+}
+
+/* ------------------------------------------------------------------------ */
+/* Calibration and scales                                                   */
+/* ------------------------------------------------------------------------ */
+
+/* [FP8-KV] calibrator: the observed absolute maximum of a BF16 tensor. */
+float orc_absmax_bf16(const uint16_t* x, int64_t n) {
+  float m = 0.0f;
+  for (int64_t i = 0; i < n; i++) {
+    float a = fabsf(bf16_to_f32(x[i]));
+    if (a > m) m = a;
+  }
+  return m;
+}
+
+/* [FP8-KV]: scale = max(observed_absolute_max * 1.05 / 448, 1e-12), evaluated
+ * in fp32 left to right. */
+float orc_fp8_scale(float amax) {
+  float s = (amax * 1.05f) / 448.0f;
+  if (s < 1e-12f) s = 1e-12f;
+  return s;
+}
+
+/* NVFP4 per-tensor scale g = absmax / (448 * 6), fp32 (448 * 6 = 2688 exactly). */
+float orc_nvfp4_global_scale(float amax) { return amax / (448.0f * 6.0f); }
+
+/* ------------------------------------------------------------------------ */
+/* Paged cache layout                                                       */
+/* ------------------------------------------------------------------------ */
+/*
+ * K and V are separate buffers with identical layout.  A cache slot is
+ * block * 16 + offset.  For head h of block blk the "head page" holds the 16
+ * tokens of that block for that head:
+ *   BF16 : uint16 [blk][h][16][D]
+ *   FP8  : uint8  [blk][h][16][D]   (E4M3 codes)
+ *   NVFP4: bytes  [blk][h][ 16*D/2 codes | 16*D/16 block scales ]  (9*D bytes)
+ *          codes  [16][D/2]: element 2j in the low nibble, 2j+1 in the high one
+ *          scales [16][D/16]: one E4M3 byte per 16-element block along D
+ */
+static int64_t head_page_index(int64_t blk, int h, int H) { return blk * H + h; }
+
+/* Dequantised value of element (blk, h, o, d) as the fp32 the method defines:
+ *   BF16 : the BF16 value;
+ *   FP8  : fp32(dec_e4m3(code) * s);
+ *   NVFP4: fp32(fp32(dec_e2m1(e) * dec_e4m3(sb)) * g)  (inner product exact). */
+static float dequant_elem(int fmt, const void* cache, int64_t blk, int h, int o, int d, int H,
+                          int D, float scale) {
+  int64_t hp = head_page_index(blk, h, H);
+  if (fmt == ORC_BF16) {
+    const uint16_t* c = (const uint16_t*)cache;
+    return bf16_to_f32(c[(hp * ORC_PAGE + o) * D + d]);
+  } else if (fmt == ORC_FP8) {
+    const uint8_t* c = (const uint8_t*)cache;
+    return orc_e4m3_decode(c[(hp * ORC_PAGE + o) * D + d]) * scale;
+  } else {
+    const uint8_t* base = (const uint8_t*)cache + hp * (int64_t)(9 * D);
+    uint8_t byte = base[o * (D / 2) + d / 2];
+    uint8_t e = (d % 2 == 0) ? (byte & 0xF) : (byte >> 4);
+    uint8_t sb = base[ORC_PAGE * (D / 2) + o * (D / 16) + d / 16];
+    float elem = orc_e2m1_decode(e) * orc_e4m3_decode(sb);
+    return elem * scale;
+  }
+}
+
+int64_t orc_head_page_bytes(int fmt, int D) {
+  if (fmt == ORC_BF16) return (int64_t)ORC_PAGE * D * 2;
+  if (fmt == ORC_FP8) return (int64_t)ORC_PAGE * D;
+  return (int64_t)9 * D;
+}
+
+/* Bytes of one token's K and V for H heads of width D in the given format. */
+double orc_kv_bytes_per_token(int fmt, int H, int D) {
+  double per_elem = (fmt == ORC_BF16) ? 2.0 : (fmt == ORC_FP8) ? 1.0 : 4.5 / 8.0;
+  return 2.0 * H * D * per_elem;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Quantize-on-write                                                        */
+/* ------------------------------------------------------------------------ */
+
+/* Quantize one [D] row of BF16 values into head page (blk, h) at offset o. */
+static void write_row(int fmt, const uint16_t* x, void* cache, int64_t blk, int h, int o, int H,
+                      int D, float scale) {
+  int64_t hp = head_page_index(blk, h, H);
+  if (fmt == ORC_BF16) {
+    uint16_t* c = (uint16_t*)cache;
+    for (int d = 0; d < D; d++) c[(hp * ORC_PAGE + o) * D + d] = x[d];
+  } else if (fmt == ORC_FP8) {
+    /* [FP8-KV]: code = E4M3(x / scale), fp32 division, RNE, satfinite. */
+    uint8_t* c = (uint8_t*)cache;
+    for (int d = 0; d < D; d++) {
+      float v = bf16_to_f32(x[d]) / scale;
+      c[(hp * ORC_PAGE + o) * D + d] = orc_e4m3_encode(v);
+    }
+  } else {
+    /* NVFP4, one 16-element block at a time along D. */
+    uint8_t* base = (uint8_t*)cache + hp * (int64_t)(9 * D);
+    float g = scale;
+    for (int blk16 = 0; blk16 < D / 16; blk16++) {
+      float bmax = 0.0f;
+      for (int i = 0; i < 16; i++) {
+        float a = fabsf(bf16_to_f32(x[blk16 * 16 + i]));
+        if (a > bmax) bmax = a;
+      }
+      uint8_t sb;
+      float den;
+      if (g > 0.0f) {
+        sb = orc_e4m3_encode(bmax / (6.0f * g));
+        den = orc_e4m3_decode(sb) * g;
+      } else {
+        sb = 0; /* g == 0: an all-zero tensor; every code is +0 */
+        den = 0.0f;
+      }
+      base[ORC_PAGE * (D / 2) + o * (D / 16) + blk16] = sb;
+      for (int i = 0; i < 16; i += 2) {
+        int d = blk16 * 16 + i;
+        uint8_t e0 = 0, e1 = 0;
+        if (den != 0.0f) {
+          e0 = orc_e2m1_encode(bf16_to_f32(x[d]) / den);
+          e1 = orc_e2m1_encode(bf16_to_f32(x[d + 1]) / den);
+        }
+        base[o * (D / 2) + d / 2] = (uint8_t)(e0 | (e1 << 4));
+      }
+    }
+  }
+}
+
+/* Write tokens [0, T) of k, v ([T][H][D] BF16) to the slots slot_mapping[t]
+ * (block = slot / 16, offset = slot % 16).  A negative slot skips the token.
+ * Returns 0, or -1 if a slot lies beyond the cache (nothing is written for it). */
+int orc_write(int fmt, const uint16_t* k, const uint16_t* v, int64_t T, int H, int D,
+              const int64_t* slot_mapping, int64_t num_blocks, void* k_cache, void* v_cache,
+              float k_scale, float v_scale) {
+  int rc = 0;
+  for (int64_t t = 0; t < T; t++) {
+    int64_t slot = slot_mapping[t];
+    if (slot < 0) continue;
+    int64_t blk = slot / ORC_PAGE;
+    int o = (int)(slot % ORC_PAGE);
+    if (blk >= num_blocks) {
+      rc = -1;
+      continue;
+    }
+    for (int h = 0; h < H; h++) {
+      write_row(fmt, k + (t * H + h) * D, k_cache, blk, h, o, H, D, k_scale);
+      write_row(fmt, v + (t * H + h) * D, v_cache, blk, h, o, H, D, v_scale);
+    }
+  }
+  return rc;
+}
+
+/* Dequantise the listed slots into k_out, v_out ([n][H][D] fp32). */
+int orc_dequantize(int fmt, const void* k_cache, const void* v_cache, int64_t num_blocks, int H,
+                   int D, const int64_t* slots, int64_t n, float k_scale, float v_scale,
+                   float* k_out, float* v_out) {
+  for (int64_t i = 0; i < n; i++) {
+    int64_t slot = slots[i];
+    if (slot < 0 || slot / ORC_PAGE >= num_blocks) return -1;
+    int64_t blk = slot / ORC_PAGE;
+    int o = (int)(slot % ORC_PAGE);
+    for (int h = 0; h < H; h++)
+      for (int d = 0; d < D; d++) {
+        k_out[(i * H + h) * D + d] = dequant_elem(fmt, k_cache, blk, h, o, d, H, D, k_scale);
+        v_out[(i * H + h) * D + d] = dequant_elem(fmt, v_cache, blk, h, o, d, H, D, v_scale);
+      }
+  }
+  return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Decode attention, float64                                                */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * Softmax attention of one query head over context tokens [t0, t1) of
+ * sequence b, over the dequantised cache values, in float64:
+ *   s_t = sm_scale * sum_d q_d * k_hat_{t,d}
+ *   m   = max_t s_t,   l = sum_t exp(s_t - m),   o_unnorm = sum_t exp(s_t - m) v_hat_t
+ * Token t of the sequence lives in block block_table[b][t / 16] at offset
+ * t % 16.  Query head j reads KV head j / (Hq / H).  An empty range returns
+ * m = -inf, l = 0, o_unnorm = 0.  Returns -1 if a block id is out of range.
+ */
+int orc_attention_range(int fmt, const uint16_t* q_row, const void* k_cache, const void* v_cache,
+                        int64_t num_blocks, int H, int D, const int32_t* bt_row, int kv_head,
+                        int64_t t0, int64_t t1, float k_scale, float v_scale, double sm_scale,
+                        double* o_unnorm, double* m_out, double* l_out) {
+  int64_t n = t1 - t0;
+  for (int d = 0; d < D; d++) o_unnorm[d] = 0.0;
+  if (n <= 0) {
+    *m_out = -INFINITY;
+    *l_out = 0.0;
+    return 0;
+  }
+  double* s = (double*)malloc(sizeof(double) * (size_t)n);
+  if (!s) return -2;
+  double m = -INFINITY;
+  for (int64_t t = t0; t < t1; t++) {
+    int64_t blk = bt_row[t / ORC_PAGE];
+    if (blk < 0 || blk >= num_blocks) {
+      free(s);
+      return -1;
+    }
+    int o = (int)(t % ORC_PAGE);
+    double acc = 0.0;
+    for (int d = 0; d < D; d++)
+      acc += (double)bf16_to_f32(q_row[d]) *
+             (double)dequant_elem(fmt, k_cache, blk, kv_head, o, d, H, D, k_scale);
+    s[t - t0] = sm_scale * acc;
+    if (s[t - t0] > m) m = s[t - t0];
+  }
+  double l = 0.0;
+  for (int64_t t = t0; t < t1; t++) {
+    double p = exp(s[t - t0] - m);
+    l += p;
+    int64_t blk = bt_row[t / ORC_PAGE];
+    int o = (int)(t % ORC_PAGE);
+    for (int d = 0; d < D; d++)
+      o_unnorm[d] += p * (double)dequant_elem(fmt, v_cache, blk, kv_head, o, d, H, D, v_scale);
+  }
+  free(s);
+  *m_out = m;
+  *l_out = l;
+  return 0;
+}
+
+/*
+ * Full decode step: out[b][j][:] = o_unnorm / l and lse[b][j] = m + ln(l) for
+ * every sequence b and query head j (natural log, scaled-score units).  A
+ * sequence of length 0 gives out = 0 and lse = -inf.  q is [B][Hq][D] BF16;
+ * block_table is [B][max_blocks]; out is [B][Hq][D], lse [B][Hq] (float64).
+ * If pairs is non-NULL, only the n_pairs (b, j) pairs listed in it (as
+ * pairs[2i], pairs[2i+1]) are computed; other outputs are left untouched.
+ */
+int orc_decode_attention(int fmt, const uint16_t* q, const void* k_cache, const void* v_cache,
+                         int64_t num_blocks, int H, int D, const int32_t* block_table,
+                         int max_blocks, const int32_t* seq_lens, int B, int Hq, float k_scale,
+                         float v_scale, double sm_scale, const int32_t* pairs, int64_t n_pairs,
+                         double* out, double* lse) {
+  int G = Hq / H;
+  int64_t total = pairs ? n_pairs : (int64_t)B * Hq;
+  for (int64_t i = 0; i < total; i++) {
+    int b = pairs ? pairs[2 * i] : (int)(i / Hq);
+    int j = pairs ? pairs[2 * i + 1] : (int)(i % Hq);
+    double m, l;
+    double* o = out + ((int64_t)b * Hq + j) * D;
+    int rc = orc_attention_range(fmt, q + ((int64_t)b * Hq + j) * D, k_cache, v_cache, num_blocks,
+                                 H, D, block_table + (int64_t)b * max_blocks, j / G, 0,
+                                 seq_lens[b], k_scale, v_scale, sm_scale, o, &m, &l);
+    if (rc) return rc;
+    if (l > 0.0) {
+      for (int d = 0; d < D; d++) o[d] /= l;
+      lse[(int64_t)b * Hq + j] = m + log(l);
+    } else {
+      lse[(int64_t)b * Hq + j] = -INFINITY;
+    }
+  }
+  return 0;
+}
+
+/*
+ * Merge of n partial results (o_unnorm_i, m_i, l_i) of disjoint context
+ * ranges into the full one:
+ *   M = max_i m_i,  L = sum_i exp(m_i - M) l_i,
+ *   out = sum_i exp(m_i - M) o_unnorm_i / L,  lse = M + ln L.
+ * Parts with m_i = -inf (empty ranges) contribute nothing.
+ */
+void orc_merge(int n, int D, const double* o_parts, const double* m_parts, const double* l_parts,
+               double* out, double* lse) {
+  double M = -INFINITY;
+  for (int i = 0; i < n; i++)
+    if (m_parts[i] > M) M = m_parts[i];
+  for (int d = 0; d < D; d++) out[d] = 0.0;
+  if (M == -INFINITY) {
+    *lse = -INFINITY;
+    return;
+  }
+  double L = 0.0;
+  for (int i = 0; i < n; i++) {
+    if (m_parts[i] == -INFINITY) continue;
+    double w = exp(m_parts[i] - M);
+    L += w * l_parts[i];
+    for (int d = 0; d < D; d++) out[d] += w * o_parts[(int64_t)i * D + d];
+  }
+  for (int d = 0; d < D; d++) out[d] /= L;
+  *lse = M + log(L);
+}
