@@ -1,0 +1,410 @@
+// kvq_api.cu -- the C ABI declared in include/kvq.h: argument checks, the
+// context-split plan, TMA descriptors for the paged cache, and launches.
+#include <cudaTypedefs.h>
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+
+#include <atomic>
+#include <mutex>
+
+#include "kvq.h"
+#include "kvq_internal.h"
+
+namespace {
+
+thread_local char g_err[512] = "";
+
+kvq_status fail(kvq_status s, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return s;
+}
+
+kvq_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(KVQ_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+// 0 = unknown, 1 = supported (sm_100), 2 = not supported.
+std::atomic<int> g_dev_ok[64];
+
+kvq_status check_device() {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= 64) return fail(KVQ_ERR_UNSUPPORTED, "device ordinal %d", dev);
+  int st = g_dev_ok[dev].load(std::memory_order_relaxed);
+  if (st == 0) {
+    int major = 0, minor = 0;
+    e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+    st = (major == 10 && minor == 0) ? 1 : 2;
+    g_dev_ok[dev].store(st, std::memory_order_relaxed);
+  }
+  if (st != 1) return fail(KVQ_ERR_UNSUPPORTED, "device %d is not compute capability 10.0 (B200)", dev);
+  return KVQ_OK;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+int64_t head_page_bytes(int fmt, int D) {
+  if (fmt == KVQ_FMT_BF16) return 32LL * D;
+  if (fmt == KVQ_FMT_FP8_E4M3) return 16LL * D;
+  return 9LL * D;
+}
+
+kvq_status check_cache(int32_t fmt, const kvq_cache* c) {
+  if (fmt < 0 || fmt > 2) return fail(KVQ_ERR_UNSUPPORTED, "unknown format %d", fmt);
+  if (!c) return fail(KVQ_ERR_INVALID_ARG, "cache is NULL");
+  if (c->fmt != fmt) return fail(KVQ_ERR_INVALID_ARG, "cache format %d != fmt %d", c->fmt, fmt);
+  if (c->block_size != KVQ_BLOCK_SIZE)
+    return fail(KVQ_ERR_UNSUPPORTED, "block_size %d (only 16)", c->block_size);
+  if (c->head_dim != 64 && c->head_dim != 128)
+    return fail(KVQ_ERR_UNSUPPORTED, "head_dim %d (64 or 128)", c->head_dim);
+  if (c->num_kv_heads < 1) return fail(KVQ_ERR_INVALID_ARG, "num_kv_heads %d", c->num_kv_heads);
+  if (c->num_blocks < 1 || c->num_blocks > 0x7fffffffLL)
+    return fail(KVQ_ERR_INVALID_ARG, "num_blocks %lld", (long long)c->num_blocks);
+  if (!c->k || !c->v) return fail(KVQ_ERR_INVALID_ARG, "cache k/v is NULL");
+  if (!aligned(c->k, 256) || !aligned(c->v, 256))
+    return fail(KVQ_ERR_INVALID_ARG, "cache k/v must be 256-byte aligned");
+  return KVQ_OK;
+}
+
+// ---------------------------------------------------------------- split plan
+struct Plan {
+  int G, n_groups, units, splits, pps;
+  size_t off_ml, off_o, ws_bytes;
+};
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+kvq_status make_plan(int32_t fmt, int32_t B, int32_t Hq, int32_t Hkv, int32_t D,
+                     int32_t max_seq_len, int32_t num_splits, Plan* pl) {
+  kvq::DecodeConfig cfg;
+  if (fmt < 0 || fmt > 2 || !kvq::decode_config(fmt, D, &cfg))
+    return fail(KVQ_ERR_UNSUPPORTED, "format %d / head_dim %d", fmt, D);
+  if (B < 0 || Hkv < 1 || Hq < Hkv || Hq % Hkv != 0)
+    return fail(KVQ_ERR_INVALID_ARG, "num_seqs %d, num_q_heads %d, num_kv_heads %d", B, Hq, Hkv);
+  if (max_seq_len < 0) return fail(KVQ_ERR_INVALID_ARG, "max_seq_len %d", max_seq_len);
+  if (num_splits < 0) return fail(KVQ_ERR_INVALID_ARG, "num_splits %d", num_splits);
+  pl->G = Hq / Hkv;
+  pl->n_groups = (pl->G + 7) / 8;
+  pl->units = B * Hkv * pl->n_groups;
+  const int max_pages = (max_seq_len + KVQ_BLOCK_SIZE - 1) / KVQ_BLOCK_SIZE;
+  int splits;
+  if (num_splits > 0) {
+    splits = num_splits;
+  } else {
+    const int per_sm = kvq::decode_ctas_per_sm(fmt, D);
+    const int ctas = (per_sm > 0 ? per_sm : 1) * kvq::num_sms();
+    splits = pl->units > 0 ? ctas / pl->units : 1;
+    const int by_pages = (max_pages + 2 * cfg.warps - 1) / (2 * cfg.warps);  // >= 2 pages/warp
+    if (splits > by_pages) splits = by_pages;
+  }
+  if (splits > 512) splits = 512;
+  if (splits > max_pages) splits = max_pages;
+  if (splits < 1) splits = 1;
+  int pps = (max_pages + splits - 1) / splits;
+  if (pps < 1) pps = 1;
+  splits = (max_pages + pps - 1) / pps;
+  if (splits < 1) splits = 1;
+  pl->splits = splits;
+  pl->pps = pps;
+  if (splits > 1) {
+    const size_t cnt = align_up(sizeof(unsigned) * pl->units, 256);
+    const size_t ml = align_up(sizeof(float) * 2 * 8 * (size_t)pl->units * splits, 256);
+    pl->off_ml = cnt;
+    pl->off_o = cnt + ml;
+    pl->ws_bytes = cnt + ml + sizeof(float) * 8 * (size_t)D * pl->units * splits;
+  } else {
+    pl->off_ml = pl->off_o = 0;
+    pl->ws_bytes = 0;
+  }
+  return KVQ_OK;
+}
+
+// ---------------------------------------------------------------- TMA maps
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+kvq_status encode(CUtensorMap* m, CUtensorMapDataType dt, cuuint32_t rank, void* base,
+                  const cuuint64_t* dims, const cuuint64_t* strides, const cuuint32_t* box,
+                  CUtensorMapSwizzle sw) {
+  auto fn = encode_fn();
+  if (!fn) return fail(KVQ_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  const cuuint32_t es[5] = {1, 1, 1, 1, 1};
+  CUresult r = fn(m, dt, rank, base, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(KVQ_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return KVQ_OK;
+}
+
+// Descriptors for one cache buffer: [0] = codes/values tile of a head page,
+// [1] = NVFP4 block-scale run of a head page (same as [0] otherwise).
+kvq_status make_maps(int fmt, const kvq_cache* c, void* buf, CUtensorMap* tile, CUtensorMap* sf) {
+  const cuuint64_t D = c->head_dim, H = c->num_kv_heads, nb = c->num_blocks;
+  if (fmt == KVQ_FMT_FP8_E4M3) {
+    const cuuint64_t dims[4] = {D, 16, H, nb};
+    const cuuint64_t str[3] = {D, 16 * D, 16 * D * H};
+    const cuuint32_t box[4] = {(cuuint32_t)D, 16, 1, 1};
+    kvq_status s = encode(tile, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, buf, dims, str, box,
+                          D == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B);
+    *sf = *tile;
+    return s;
+  }
+  if (fmt == KVQ_FMT_BF16) {
+    const cuuint64_t dims[4] = {D, 16, H, nb};
+    const cuuint64_t str[3] = {2 * D, 32 * D, 32 * D * H};
+    const cuuint32_t box[4] = {64, 16, 1, 1};
+    kvq_status s = encode(tile, CU_TENSOR_MAP_DATA_TYPE_UINT16, 4, buf, dims, str, box,
+                          CU_TENSOR_MAP_SWIZZLE_128B);
+    *sf = *tile;
+    return s;
+  }
+  // NVFP4: head page = 16 rows of D/2 code bytes, then 16 * D/16 scale bytes
+  const cuuint64_t dims[4] = {D / 2, 16, H, nb};
+  const cuuint64_t str[3] = {D / 2, 9 * D, 9 * D * H};
+  const cuuint32_t box[4] = {(cuuint32_t)(D / 2), 16, 1, 1};
+  kvq_status s = encode(tile, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, buf, dims, str, box,
+                        D == 64 ? CU_TENSOR_MAP_SWIZZLE_32B : CU_TENSOR_MAP_SWIZZLE_64B);
+  if (s != KVQ_OK) return s;
+  const cuuint64_t dims_s[3] = {D, H, nb};
+  const cuuint64_t str_s[2] = {9 * D, 9 * D * H};
+  const cuuint32_t box_s[3] = {(cuuint32_t)D, 1, 1};
+  return encode(sf, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, static_cast<uint8_t*>(buf) + 8 * D, dims_s,
+                str_s, box_s, CU_TENSOR_MAP_SWIZZLE_NONE);
+}
+
+}  // namespace
+
+namespace kvq {
+int num_sms() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 148;
+  return n;
+}
+}  // namespace kvq
+
+extern "C" {
+
+const char* kvq_status_string(kvq_status s) {
+  switch (s) {
+    case KVQ_OK: return "ok";
+    case KVQ_ERR_INVALID_ARG: return "invalid argument";
+    case KVQ_ERR_UNSUPPORTED: return "unsupported";
+    case KVQ_ERR_WORKSPACE: return "workspace missing or too small";
+    case KVQ_ERR_CUDA: return "CUDA error";
+  }
+  return "unknown status";
+}
+
+const char* kvq_last_error(void) { return g_err; }
+
+kvq_status kv_cache_bytes(int32_t fmt, int64_t num_blocks, int32_t num_kv_heads,
+                          int32_t head_dim, int64_t* bytes) {
+  if (fmt < 0 || fmt > 2) return fail(KVQ_ERR_UNSUPPORTED, "unknown format %d", fmt);
+  if (head_dim != 64 && head_dim != 128) return fail(KVQ_ERR_UNSUPPORTED, "head_dim %d", head_dim);
+  if (num_blocks < 0 || num_kv_heads < 1 || !bytes)
+    return fail(KVQ_ERR_INVALID_ARG, "num_blocks/num_kv_heads/bytes");
+  *bytes = num_blocks * num_kv_heads * head_page_bytes(fmt, head_dim);
+  return KVQ_OK;
+}
+
+kvq_status kv_scale_from_absmax(int32_t fmt, float amax, float* scale) {
+  if (fmt < 0 || fmt > 2) return fail(KVQ_ERR_UNSUPPORTED, "unknown format %d", fmt);
+  if (!scale) return fail(KVQ_ERR_INVALID_ARG, "scale is NULL");
+  if (!(amax >= 0.0f) || isinf(amax)) return fail(KVQ_ERR_INVALID_ARG, "amax must be finite, >= 0");
+  volatile float a = amax;  // keep the fp32 evaluation order literal
+  if (fmt == KVQ_FMT_FP8_E4M3) {
+    volatile float t = a * 1.05f;
+    float s = t / 448.0f;
+    if (s < 1e-12f) s = 1e-12f;
+    *scale = s;
+  } else if (fmt == KVQ_FMT_NVFP4) {
+    *scale = a / 2688.0f;
+  } else {
+    *scale = 1.0f;
+  }
+  return KVQ_OK;
+}
+
+kvq_status kv_scale_from_absmax_device(int32_t fmt, const float* d_amax, float* d_scale,
+                                       kvq_stream stream) {
+  if (fmt < 0 || fmt > 2) return fail(KVQ_ERR_UNSUPPORTED, "unknown format %d", fmt);
+  if (!d_amax || !d_scale) return fail(KVQ_ERR_INVALID_ARG, "d_amax/d_scale is NULL");
+  kvq_status s = check_device();
+  if (s != KVQ_OK) return s;
+  cudaError_t e = kvq::launch_scale(fmt, d_amax, d_scale, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? KVQ_OK : cuda_fail(e, "scale kernel");
+}
+
+kvq_status kv_calibrate_absmax(const void* x, int64_t n, float* d_amax, kvq_stream stream) {
+  if (n < 0) return fail(KVQ_ERR_INVALID_ARG, "n %lld", (long long)n);
+  if (!d_amax || !aligned(d_amax, 4)) return fail(KVQ_ERR_INVALID_ARG, "d_amax NULL or misaligned");
+  if (n > 0 && (!x || !aligned(x, 2))) return fail(KVQ_ERR_INVALID_ARG, "x NULL or misaligned");
+  kvq_status s = check_device();
+  if (s != KVQ_OK) return s;
+  cudaError_t e = kvq::launch_absmax(static_cast<const uint16_t*>(x), n, d_amax,
+                                     static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? KVQ_OK : cuda_fail(e, "absmax kernel");
+}
+
+kvq_status kv_quantize_write(int32_t fmt, const void* k, const void* v, int64_t num_tokens,
+                             const int64_t* slot_mapping, const int32_t* block_table,
+                             int32_t num_seqs, int32_t max_blocks, const kvq_cache* cache,
+                             const float* d_k_scale, const float* d_v_scale, int32_t* d_err,
+                             kvq_stream stream) {
+  kvq_status s = check_cache(fmt, cache);
+  if (s != KVQ_OK) return s;
+  if (num_tokens < 0) return fail(KVQ_ERR_INVALID_ARG, "num_tokens %lld", (long long)num_tokens);
+  if (num_tokens > 0) {
+    if (!k || !v || !aligned(k, 16) || !aligned(v, 16))
+      return fail(KVQ_ERR_INVALID_ARG, "k/v NULL or not 16-byte aligned");
+    if (!slot_mapping) return fail(KVQ_ERR_INVALID_ARG, "slot_mapping is NULL");
+  }
+  if (block_table && (num_seqs < 1 || max_blocks < 1))
+    return fail(KVQ_ERR_INVALID_ARG, "block_table given with num_seqs %d, max_blocks %d",
+                num_seqs, max_blocks);
+  if (fmt != KVQ_FMT_BF16 && (!d_k_scale || !d_v_scale))
+    return fail(KVQ_ERR_INVALID_ARG, "quantized formats need d_k_scale and d_v_scale");
+  s = check_device();
+  if (s != KVQ_OK) return s;
+  kvq::QuantParams p;
+  p.k = static_cast<const uint16_t*>(k);
+  p.v = static_cast<const uint16_t*>(v);
+  p.T = num_tokens;
+  p.H = cache->num_kv_heads;
+  p.D = cache->head_dim;
+  p.slot_mapping = slot_mapping;
+  p.block_table = block_table;
+  p.num_seqs = num_seqs;
+  p.max_blocks = max_blocks;
+  p.num_blocks = cache->num_blocks;
+  p.kc = static_cast<uint8_t*>(cache->k);
+  p.vc = static_cast<uint8_t*>(cache->v);
+  p.k_scale = d_k_scale;
+  p.v_scale = d_v_scale;
+  p.d_err = d_err;
+  cudaError_t e = kvq::launch_quantize(fmt, p, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? KVQ_OK : cuda_fail(e, "quantize kernel");
+}
+
+kvq_status kv_decode_workspace_size(int32_t fmt, int32_t num_seqs, int32_t num_q_heads,
+                                    int32_t num_kv_heads, int32_t head_dim, int32_t max_seq_len,
+                                    int32_t num_splits, size_t* bytes) {
+  if (!bytes) return fail(KVQ_ERR_INVALID_ARG, "bytes is NULL");
+  kvq_status s = check_device();
+  if (s != KVQ_OK) return s;
+  Plan pl;
+  s = make_plan(fmt, num_seqs, num_q_heads, num_kv_heads, head_dim, max_seq_len, num_splits, &pl);
+  if (s != KVQ_OK) return s;
+  *bytes = pl.ws_bytes;
+  return KVQ_OK;
+}
+
+kvq_status kv_decode_attention(int32_t fmt, const void* q, const kvq_cache* cache,
+                               const int32_t* block_table, int32_t max_blocks,
+                               const int32_t* seq_lens, int32_t num_seqs, int32_t num_q_heads,
+                               int32_t max_seq_len, int32_t num_splits, const float* d_k_scale,
+                               const float* d_v_scale, float sm_scale, float* out, float* lse,
+                               void* workspace, size_t workspace_bytes, int32_t* d_err,
+                               kvq_stream stream) {
+  kvq_status s = check_cache(fmt, cache);
+  if (s != KVQ_OK) return s;
+  const int D = cache->head_dim, Hkv = cache->num_kv_heads;
+  if (num_seqs < 0) return fail(KVQ_ERR_INVALID_ARG, "num_seqs %d", num_seqs);
+  if (num_seqs == 0) return KVQ_OK;
+  if (!q || !aligned(q, 2)) return fail(KVQ_ERR_INVALID_ARG, "q NULL or misaligned");
+  if (!block_table || !seq_lens) return fail(KVQ_ERR_INVALID_ARG, "block_table/seq_lens NULL");
+  if (!out || !aligned(out, 4)) return fail(KVQ_ERR_INVALID_ARG, "out NULL or misaligned");
+  if (max_blocks < 1) return fail(KVQ_ERR_INVALID_ARG, "max_blocks %d", max_blocks);
+  if (max_seq_len < 0 || (int64_t)max_seq_len > (int64_t)max_blocks * KVQ_BLOCK_SIZE)
+    return fail(KVQ_ERR_INVALID_ARG, "max_seq_len %d exceeds max_blocks * 16", max_seq_len);
+  if (fmt != KVQ_FMT_BF16 && (!d_k_scale || !d_v_scale))
+    return fail(KVQ_ERR_INVALID_ARG, "quantized formats need d_k_scale and d_v_scale");
+  if (sm_scale == 0.0f) sm_scale = 1.0f / sqrtf((float)D);
+  if (!isfinite(sm_scale)) return fail(KVQ_ERR_INVALID_ARG, "sm_scale not finite");
+  s = check_device();
+  if (s != KVQ_OK) return s;
+  Plan pl;
+  s = make_plan(fmt, num_seqs, num_q_heads, Hkv, D, max_seq_len, num_splits, &pl);
+  if (s != KVQ_OK) return s;
+  if (Hkv * pl.n_groups > 65535 || num_seqs > 65535)
+    return fail(KVQ_ERR_UNSUPPORTED, "grid too large (heads %d, seqs %d)", Hkv, num_seqs);
+  if (pl.ws_bytes > 0) {
+    if (!workspace || !aligned(workspace, 256))
+      return fail(KVQ_ERR_WORKSPACE, "workspace NULL or not 256-byte aligned (%zu bytes needed)",
+                  pl.ws_bytes);
+    if (workspace_bytes < pl.ws_bytes)
+      return fail(KVQ_ERR_WORKSPACE, "workspace %zu bytes < %zu needed", workspace_bytes,
+                  pl.ws_bytes);
+  }
+  CUtensorMap maps[4];
+  s = make_maps(fmt, cache, cache->k, &maps[0], &maps[2]);
+  if (s != KVQ_OK) return s;
+  s = make_maps(fmt, cache, cache->v, &maps[1], &maps[3]);
+  if (s != KVQ_OK) return s;
+
+  kvq::DecodeParams p;
+  p.q = static_cast<const uint16_t*>(q);
+  p.block_table = block_table;
+  p.seq_lens = seq_lens;
+  p.k_scale = d_k_scale;
+  p.v_scale = d_v_scale;
+  p.out = out;
+  p.lse = lse;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  p.ws_cnt = pl.ws_bytes ? reinterpret_cast<unsigned*>(ws) : nullptr;
+  p.ws_ml = pl.ws_bytes ? reinterpret_cast<float*>(ws + pl.off_ml) : nullptr;
+  p.ws_o = pl.ws_bytes ? reinterpret_cast<float*>(ws + pl.off_o) : nullptr;
+  p.d_err = d_err;
+  p.num_blocks = cache->num_blocks;
+  p.max_blocks = max_blocks;
+  p.B = num_seqs;
+  p.Hq = num_q_heads;
+  p.Hkv = Hkv;
+  p.G = pl.G;
+  p.n_groups = pl.n_groups;
+  p.max_seq_len = max_seq_len;
+  p.num_splits = pl.splits;
+  p.pages_per_split = pl.pps;
+  p.sm_scale = sm_scale;
+  cudaError_t e = kvq::launch_decode(fmt, D, maps, p, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? KVQ_OK : cuda_fail(e, "decode kernel");
+}
+
+kvq_status kv_dequantize(int32_t fmt, const kvq_cache* cache, const int64_t* slots, int64_t n,
+                         const float* d_k_scale, const float* d_v_scale, float* k_out,
+                         float* v_out, int32_t* d_err, kvq_stream stream) {
+  kvq_status s = check_cache(fmt, cache);
+  if (s != KVQ_OK) return s;
+  if (n < 0) return fail(KVQ_ERR_INVALID_ARG, "n %lld", (long long)n);
+  if (n > 0 && (!slots || !k_out || !v_out || !aligned(k_out, 16) || !aligned(v_out, 16)))
+    return fail(KVQ_ERR_INVALID_ARG, "slots/k_out/v_out NULL or outputs not 16-byte aligned");
+  if (fmt != KVQ_FMT_BF16 && (!d_k_scale || !d_v_scale))
+    return fail(KVQ_ERR_INVALID_ARG, "quantized formats need d_k_scale and d_v_scale");
+  s = check_device();
+  if (s != KVQ_OK) return s;
+  cudaError_t e = kvq::launch_dequantize(
+      fmt, static_cast<const uint8_t*>(cache->k), static_cast<const uint8_t*>(cache->v),
+      cache->num_blocks, cache->num_kv_heads, cache->head_dim, slots, n, d_k_scale, d_v_scale,
+      k_out, v_out, d_err, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? KVQ_OK : cuda_fail(e, "dequantize kernel");
+}
+
+}  // extern "C"

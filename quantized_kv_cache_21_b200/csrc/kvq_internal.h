@@ -1,0 +1,74 @@
+// kvq_internal.h -- launch interfaces shared by the C-ABI layer and the
+// kernel translation units (host side only).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace kvq {
+
+struct DecodeParams {
+  const uint16_t* q;          // [B][Hq][D] bf16
+  const int32_t* block_table; // [B][max_blocks]
+  const int32_t* seq_lens;    // [B]
+  const float* k_scale;       // device scalar (FP8: s, NVFP4: g); unused for BF16
+  const float* v_scale;
+  float* out;                 // [B][Hq][D]
+  float* lse;                 // [B][Hq] or null
+  float* ws_o;                // [units][splits][8][D]
+  float* ws_ml;               // [units][splits][8][2]
+  unsigned* ws_cnt;           // [units]
+  int* d_err;
+  int64_t num_blocks;
+  int max_blocks;
+  int B, Hq, Hkv, G, n_groups;
+  int max_seq_len;
+  int num_splits, pages_per_split;
+  float sm_scale;
+};
+
+struct DecodeConfig {
+  int warps;        // warps per CTA
+  int stages;       // shared-memory stages per warp
+  int stage_bytes;  // bytes per stage
+  size_t smem_bytes;
+};
+
+// Per-(format, head_dim) kernel configuration; false if unsupported.
+bool decode_config(int fmt, int D, DecodeConfig* cfg);
+// Resident CTAs per SM of the decode kernel (occupancy), 0 on error.
+int decode_ctas_per_sm(int fmt, int D);
+// Launch the decode kernel on a (splits, Hkv*n_groups, B) grid.
+cudaError_t launch_decode(int fmt, int D, const CUtensorMap* maps, const DecodeParams& p,
+                          cudaStream_t stream);
+
+struct QuantParams {
+  const uint16_t* k;
+  const uint16_t* v;
+  int64_t T;
+  int H, D;
+  const int64_t* slot_mapping;
+  const int32_t* block_table;  // null: physical slots
+  int num_seqs, max_blocks;
+  int64_t num_blocks;
+  uint8_t* kc;
+  uint8_t* vc;
+  const float* k_scale;
+  const float* v_scale;
+  int* d_err;
+};
+cudaError_t launch_quantize(int fmt, const QuantParams& p, cudaStream_t stream);
+
+cudaError_t launch_dequantize(int fmt, const uint8_t* kc, const uint8_t* vc, int64_t num_blocks,
+                              int H, int D, const int64_t* slots, int64_t n, const float* ks,
+                              const float* vs, float* ko, float* vo, int* d_err,
+                              cudaStream_t stream);
+
+cudaError_t launch_absmax(const uint16_t* x, int64_t n, float* d_amax, cudaStream_t stream);
+cudaError_t launch_scale(int fmt, const float* d_amax, float* d_scale, cudaStream_t stream);
+
+int num_sms();
+
+}  // namespace kvq

@@ -1,0 +1,72 @@
+"""The C-ABI library: it builds for sm_100a, loads, exports every function the
+public header declares, and its pure host functions agree with the oracle.
+No kernel is launched here (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle
+import quantized_kv_cache_21_b200 as kvq
+from quantized_kv_cache_21_b200 import build as kbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def header_functions():
+    text = open(os.path.join(ROOT, "include", "kvq.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return re.findall(r"^\s*(?:const\s+char\s*\*|kvq_status)\s+(\w+)\s*\(", text, flags=re.M)
+
+
+@pytest.fixture(scope="module")
+def L():
+    kbuild.build()
+    return kvq.lib()
+
+
+def test_header_symbols_are_exported(L):
+    names = header_functions()
+    assert len(names) >= 10
+    assert set(names) == set(kvq.EXPORTS)
+    for n in names:
+        assert hasattr(L, n), n
+    # the oracle is not linked into the product library
+    assert not hasattr(ctypes.CDLL(kbuild.LIB), "orc_e4m3_encode")
+
+
+def test_library_is_sm100a_only():
+    # the fatbin carries sm_100a SASS only: nvcc was asked for that gencode
+    assert kbuild.ARCH == ["-gencode", "arch=compute_100a,code=sm_100a"]
+
+
+def test_status_strings(L):
+    assert L.kvq_status_string(0) == b"ok"
+    assert b"invalid" in L.kvq_status_string(1)
+
+
+def test_cache_bytes_match_oracle_layout(L):
+    for fmt in ("bf16", "fp8", "nvfp4"):
+        for D in (64, 128):
+            got = kvq.kv_cache_bytes(fmt, 37, 3, D)
+            assert got == 37 * 3 * oracle.head_page_bytes(fmt, D)
+    with pytest.raises(kvq.KvqError):
+        kvq.kv_cache_bytes("fp8", 4, 2, 96)
+    with pytest.raises(kvq.KvqError):
+        kvq.kv_cache_bytes(7, 4, 2, 64)
+
+
+def test_host_scale_matches_oracle_bit_exact(L):
+    rng = np.random.default_rng(0)
+    amax = np.concatenate([[0.0, 1e-15, 1e-9, 1.0, 448.0, 2688.0, 72.25],
+                           rng.lognormal(0, 4, 2000)]).astype(np.float32)
+    for a in amax:
+        assert np.float32(kvq.kv_scale_from_absmax("fp8", a)) == np.float32(oracle.fp8_scale(a))
+        assert (np.float32(kvq.kv_scale_from_absmax("nvfp4", a))
+                == np.float32(oracle.nvfp4_global_scale(a)))
+        assert kvq.kv_scale_from_absmax("bf16", a) == 1.0
+    for bad in (-1.0, float("nan"), float("inf")):
+        with pytest.raises(kvq.KvqError):
+            kvq.kv_scale_from_absmax("fp8", bad)

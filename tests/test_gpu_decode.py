@@ -1,0 +1,162 @@
+"""GPU parity of the fused-dequant decode attention against the float64 oracle
+(out within 2e-3 max-abs, lse within 1e-5 relative), over formats, head dims,
+GQA ratios, ragged lengths, forced and automatic context splits, and the
+method's degenerate cases; plus the device-side error reporting."""
+import numpy as np
+import pytest
+import torch
+
+import quantized_kv_cache_21_b200 as kvq
+from quantized_kv_cache_21_b200 import workloads as wl
+
+from gpu_common import DEV, Case, assert_attention_close, dev_scalar, new_err
+
+pytestmark = pytest.mark.gpu
+
+FMTS = ["bf16", "fp8", "nvfp4"]
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("splits", [0, 1, 5])
+def test_ragged_batch(fmt, D, splits):
+    c = Case(fmt, 5, 2, 16, D, [1, 15, 16, 17, 1001], seed=1000 + D, factor=16.0)
+    out, lse = c.decode(num_splits=splits)
+    assert int(c.err.item()) == 0
+    assert_attention_close(out, lse, *c.reference())
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+@pytest.mark.parametrize("G", [1, 4, 8, 16])
+def test_gqa_ratios(fmt, G):
+    Hkv = 2
+    c = Case(fmt, 2, Hkv, Hkv * G, 128, [333, 64], seed=2000 + G)
+    out, lse = c.decode()
+    assert_attention_close(out, lse, *c.reference())
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+def test_long_context_many_splits(fmt):
+    c = Case(fmt, 1, 1, 8, 64, [20000], seed=3001, factor=16.0)
+    for splits in (0, 3, 97):
+        out, lse = c.decode(num_splits=splits)
+        assert_attention_close(out, lse, *c.reference())
+
+
+def test_tiny_fp8_workload():
+    """1 sequence x 1024 tokens, 2 KV heads, GQA 4, D 64, two outlier channels
+    per head x20, blocks in order."""
+    w = wl.WORKLOADS["tiny-fp8-1k"]
+    c = Case("fp8", w.B, w.Hkv, w.Hq, w.D, [w.seq_len], seed=w.seed, permuted=False,
+             factor=w.outlier_factor, outliers_per_head=2)
+    out, lse = c.decode()
+    e_out, e_lse = assert_attention_close(out, lse, *c.reference())
+    assert e_out < 5e-4
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+def test_empty_and_single_token(fmt):
+    c = Case(fmt, 3, 2, 8, 64, [0, 1, 0], seed=4000)
+    out, lse = c.decode()
+    ref_out, ref_lse = c.reference()
+    assert_attention_close(out, lse, ref_out, ref_lse)
+    assert np.all(np.isneginf(lse[0])) and np.all(out[0] == 0)
+    assert np.all(np.isneginf(lse[2])) and np.all(out[2] == 0)
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+def test_all_sequences_empty(fmt):
+    c = Case(fmt, 2, 1, 8, 128, [0, 0], seed=4100)
+    out, lse = c.decode(max_seq_len=0)
+    assert np.all(out == 0) and np.all(np.isneginf(lse))
+
+
+@pytest.mark.parametrize("fmt", ["fp8", "nvfp4", "bf16"])
+def test_nan_bytes_in_unwritten_slots(fmt):
+    """Pages filled with 0xFF (NaN for E4M3 and BF16) before the write: the
+    masked tail of a partial last page must not leak into the result."""
+    c = Case(fmt, 2, 2, 8, 128, [37, 250], seed=4200, fill=0xFF)
+    out, lse = c.decode(num_splits=2)
+    assert_attention_close(out, lse, *c.reference())
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+def test_zero_query_is_uniform(fmt):
+    c = Case(fmt, 1, 1, 8, 64, [300], seed=4300)
+    c.q[:] = 0
+    c.d_q.zero_()
+    out, lse = c.decode(num_splits=3)
+    ref_out, ref_lse = c.reference()
+    assert_attention_close(out, lse, ref_out, ref_lse)
+    np.testing.assert_allclose(lse, np.log(300), rtol=1e-6)
+
+
+def test_identical_heads_and_determinism():
+    c = Case("fp8", 2, 2, 16, 128, [777, 500], seed=4400)
+    c.q[:, 1] = c.q[:, 0]
+    c.d_q[:, 1] = c.d_q[:, 0]
+    a_out, a_lse = c.decode()
+    b_out, b_lse = c.decode()
+    assert np.array_equal(a_out, b_out) and np.array_equal(a_lse, b_lse)
+    assert np.array_equal(a_out[:, 0], a_out[:, 1])
+
+
+def test_page_placement_is_invisible():
+    """Same tokens at different physical blocks: bit-identical output."""
+    a = Case("nvfp4", 2, 2, 16, 64, [300, 129], seed=4500, permuted=False)
+    b = Case("nvfp4", 2, 2, 16, 64, [300, 129], seed=4500, permuted=True)
+    oa, la = a.decode(num_splits=2)
+    ob, lb = b.decode(num_splits=2)
+    assert np.array_equal(oa, ob) and np.array_equal(la, lb)
+
+
+def test_custom_sm_scale():
+    c = Case("fp8", 1, 2, 8, 64, [200], seed=4600)
+    out, lse = c.decode(sm_scale=0.05)
+    assert_attention_close(out, lse, *c.reference(sm_scale=0.05))
+
+
+def test_bad_block_id_and_seq_len_are_reported():
+    c = Case("fp8", 2, 1, 8, 64, [40, 40], seed=4700)
+    bad = c.d_bt.clone()
+    bad[0, 1] = c.num_blocks + 5
+    ws = kvq.new_workspace(kvq.kv_decode_workspace_size("fp8", 2, 8, 1, 64, 48, 0))
+    out = torch.empty(2, 8, 64, device=DEV)
+    lse = torch.empty(2, 8, device=DEV)
+    err = new_err()
+    kvq.kv_decode_attention("fp8", c.d_q, c.cache, bad, c.d_lens, 48, c.d_ks, c.d_vs, out, lse,
+                            ws, err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == kvq.DERR_BLOCK_ID
+    # sequence 1 is untouched by the bad entry of sequence 0
+    ref_out, ref_lse = c.reference()
+    assert np.abs(out[1].cpu().numpy() - ref_out[1]).max() < 2e-3
+    # a length beyond max_seq_len
+    err.zero_()
+    lens = c.d_lens.clone()
+    lens[1] = 47
+    kvq.kv_decode_attention("fp8", c.d_q, c.cache, c.d_bt, lens, 40, c.d_ks, c.d_vs, out, lse,
+                            ws, err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == kvq.DERR_SEQ_LEN
+    # a bad scale on the device
+    err.zero_()
+    kvq.kv_decode_attention("fp8", c.d_q, c.cache, c.d_bt, c.d_lens, 48, dev_scalar(0.0), c.d_vs,
+                            out, lse, ws, err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == kvq.DERR_SCALE
+
+
+def test_host_side_errors():
+    c = Case("fp8", 1, 1, 8, 64, [1000], seed=4800)
+    need = kvq.kv_decode_workspace_size("fp8", 1, 8, 1, 64, 1008, 0)
+    assert need > 0
+    out = torch.empty(1, 8, 64, device=DEV)
+    with pytest.raises(kvq.KvqError, match="workspace"):
+        kvq.kv_decode_attention("fp8", c.d_q, c.cache, c.d_bt, c.d_lens, 1008, c.d_ks, c.d_vs,
+                                out, None, kvq.new_workspace(need - 256 if need > 512 else 0))
+    with pytest.raises(kvq.KvqError, match="max_seq_len"):
+        kvq.kv_decode_attention("fp8", c.d_q, c.cache, c.d_bt, c.d_lens, 1009, c.d_ks, c.d_vs,
+                                out, None, None)
+    with pytest.raises(kvq.KvqError):  # GQA ratio must divide
+        kvq.kv_decode_workspace_size("fp8", 1, 7, 2, 64, 100, 0)
