@@ -161,9 +161,10 @@ kvq_status kv_quantize_write(int32_t fmt, const void* k, const void* v, int64_t 
                              kvq_stream stream);
 
 /* Workspace bytes kv_decode_attention needs for this problem size (0 when it
- * needs none).  num_splits: 0 = let the library choose the context split
- * from the SM count; > 0 forces that split count.  The same arguments must be
- * given to kv_decode_attention. */
+ * needs none).  num_splits: 0 = let the library spread the context over the
+ * SMs (the usual choice); > 0 cuts every (sequence, KV head) into about that
+ * many pieces, each on its own CTA, merged by log-sum-exp.  The same
+ * arguments must be given to kv_decode_attention. */
 kvq_status kv_decode_workspace_size(int32_t fmt, int32_t num_seqs, int32_t num_q_heads,
                                     int32_t num_kv_heads, int32_t head_dim, int32_t max_seq_len,
                                     int32_t num_splits, size_t* bytes);

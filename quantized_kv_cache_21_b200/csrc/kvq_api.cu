@@ -73,10 +73,13 @@ kvq_status check_cache(int32_t fmt, const kvq_cache* c) {
   return KVQ_OK;
 }
 
-// ---------------------------------------------------------------- split plan
+// ---------------------------------------------------------------- work plan
+// The decode work is the virtual page space units x pmax (unit = sequence, KV
+// head, group of 8 query heads), cut evenly over `ctas` persistent CTAs.  A
+// unit that straddles CTAs is finished by a merge of its per-CTA partials.
 struct Plan {
-  int G, n_groups, units, splits, pps;
-  size_t off_ml, off_o, ws_bytes;
+  int G, n_groups, units, pmax, ctas;
+  size_t off_part, ws_bytes;
 };
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -92,35 +95,34 @@ kvq_status make_plan(int32_t fmt, int32_t B, int32_t Hq, int32_t Hkv, int32_t D,
   if (num_splits < 0) return fail(KVQ_ERR_INVALID_ARG, "num_splits %d", num_splits);
   pl->G = Hq / Hkv;
   pl->n_groups = (pl->G + 7) / 8;
-  pl->units = B * Hkv * pl->n_groups;
-  const int max_pages = (max_seq_len + KVQ_BLOCK_SIZE - 1) / KVQ_BLOCK_SIZE;
-  int splits;
-  if (num_splits > 0) {
-    splits = num_splits;
+  const int64_t units = (int64_t)B * Hkv * pl->n_groups;
+  if (units > 0x7fffffff) return fail(KVQ_ERR_UNSUPPORTED, "too many (sequence, head) units");
+  pl->units = (int)units;
+  pl->pmax = (max_seq_len + KVQ_BLOCK_SIZE - 1) / KVQ_BLOCK_SIZE;
+  const int64_t V = units * pl->pmax;
+  const int sms = kvq::num_sms();
+  int64_t ctas;
+  if (V == 0) {
+    ctas = units < sms ? units : sms;
+  } else if (num_splits > 0) {
+    ctas = units * num_splits;
   } else {
-    const int per_sm = kvq::decode_ctas_per_sm(fmt, D);
-    const int ctas = (per_sm > 0 ? per_sm : 1) * kvq::num_sms();
-    splits = pl->units > 0 ? ctas / pl->units : 1;
-    const int by_pages = (max_pages + 2 * cfg.warps - 1) / (2 * cfg.warps);  // >= 2 pages/warp
-    if (splits > by_pages) splits = by_pages;
+    ctas = V / (2 * cfg.warps);  // at least two pages per consumer warp
+    if (ctas > sms) ctas = sms;
   }
-  if (splits > 512) splits = 512;
-  if (splits > max_pages) splits = max_pages;
-  if (splits < 1) splits = 1;
-  int pps = (max_pages + splits - 1) / splits;
-  if (pps < 1) pps = 1;
-  splits = (max_pages + pps - 1) / pps;
-  if (splits < 1) splits = 1;
-  pl->splits = splits;
-  pl->pps = pps;
-  if (splits > 1) {
-    const size_t cnt = align_up(sizeof(unsigned) * pl->units, 256);
-    const size_t ml = align_up(sizeof(float) * 2 * 8 * (size_t)pl->units * splits, 256);
-    pl->off_ml = cnt;
-    pl->off_o = cnt + ml;
-    pl->ws_bytes = cnt + ml + sizeof(float) * 8 * (size_t)D * pl->units * splits;
+  if (V > 0 && ctas > V) ctas = V;
+  if (ctas > 4096) ctas = 4096;
+  if (ctas < 1) ctas = 1;
+  pl->ctas = (int)ctas;
+  // A unit that straddles CTAs is finished from per-CTA partials (one slot
+  // per (unit, CTA) pair) with an arrival counter per unit.
+  bool spans = false;
+  if (V > 0 && ctas > 1) spans = !(ctas <= units && units % ctas == 0);
+  if (spans) {
+    pl->off_part = align_up(sizeof(unsigned) * (size_t)units, 256);
+    pl->ws_bytes = pl->off_part + sizeof(float) * (size_t)cfg.part_floats * (units + ctas);
   } else {
-    pl->off_ml = pl->off_o = 0;
+    pl->off_part = 0;
     pl->ws_bytes = 0;
   }
   return KVQ_OK;
@@ -329,7 +331,8 @@ kvq_status kv_decode_attention(int32_t fmt, const void* q, const kvq_cache* cach
   const int D = cache->head_dim, Hkv = cache->num_kv_heads;
   if (num_seqs < 0) return fail(KVQ_ERR_INVALID_ARG, "num_seqs %d", num_seqs);
   if (num_seqs == 0) return KVQ_OK;
-  if (!q || !aligned(q, 2)) return fail(KVQ_ERR_INVALID_ARG, "q NULL or misaligned");
+  if (!q || !aligned(q, 16)) return fail(KVQ_ERR_INVALID_ARG, "q NULL or not 16-byte aligned");
+  if (!aligned(out, 16)) return fail(KVQ_ERR_INVALID_ARG, "out must be 16-byte aligned");
   if (!block_table || !seq_lens) return fail(KVQ_ERR_INVALID_ARG, "block_table/seq_lens NULL");
   if (!out || !aligned(out, 4)) return fail(KVQ_ERR_INVALID_ARG, "out NULL or misaligned");
   if (max_blocks < 1) return fail(KVQ_ERR_INVALID_ARG, "max_blocks %d", max_blocks);
@@ -344,8 +347,6 @@ kvq_status kv_decode_attention(int32_t fmt, const void* q, const kvq_cache* cach
   Plan pl;
   s = make_plan(fmt, num_seqs, num_q_heads, Hkv, D, max_seq_len, num_splits, &pl);
   if (s != KVQ_OK) return s;
-  if (Hkv * pl.n_groups > 65535 || num_seqs > 65535)
-    return fail(KVQ_ERR_UNSUPPORTED, "grid too large (heads %d, seqs %d)", Hkv, num_seqs);
   if (pl.ws_bytes > 0) {
     if (!workspace || !aligned(workspace, 256))
       return fail(KVQ_ERR_WORKSPACE, "workspace NULL or not 256-byte aligned (%zu bytes needed)",
@@ -370,8 +371,7 @@ kvq_status kv_decode_attention(int32_t fmt, const void* q, const kvq_cache* cach
   p.lse = lse;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   p.ws_cnt = pl.ws_bytes ? reinterpret_cast<unsigned*>(ws) : nullptr;
-  p.ws_ml = pl.ws_bytes ? reinterpret_cast<float*>(ws + pl.off_ml) : nullptr;
-  p.ws_o = pl.ws_bytes ? reinterpret_cast<float*>(ws + pl.off_o) : nullptr;
+  p.ws_part = pl.ws_bytes ? reinterpret_cast<float*>(ws + pl.off_part) : nullptr;
   p.d_err = d_err;
   p.num_blocks = cache->num_blocks;
   p.max_blocks = max_blocks;
@@ -380,11 +380,11 @@ kvq_status kv_decode_attention(int32_t fmt, const void* q, const kvq_cache* cach
   p.Hkv = Hkv;
   p.G = pl.G;
   p.n_groups = pl.n_groups;
+  p.units = pl.units;
+  p.pmax = pl.pmax;
   p.max_seq_len = max_seq_len;
-  p.num_splits = pl.splits;
-  p.pages_per_split = pl.pps;
   p.sm_scale = sm_scale;
-  cudaError_t e = kvq::launch_decode(fmt, D, maps, p, static_cast<cudaStream_t>(stream));
+  cudaError_t e = kvq::launch_decode(fmt, D, maps, p, pl.ctas, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? KVQ_OK : cuda_fail(e, "decode kernel");
 }
 

@@ -12,14 +12,19 @@
 // registers, so the step time follows the compressed bytes.
 //
 // Design (one launch per decode step):
-//   * Grid (split, KV head x head group, sequence).  A CTA owns a contiguous
-//     range of 16-token pages of one (sequence, KV head); its warps take the
-//     range's pages round-robin.
-//   * Each warp streams its pages through a private ring of shared-memory
-//     stages filled by TMA tensor copies (one per K/V tile, swizzled so the
-//     fragment reads below are bank-conflict free), completion tracked by one
-//     mbarrier per stage.  No other warp touches the ring, so there is no
-//     CTA-wide synchronisation in the loop.
+//   * Work = the virtual page space units x pmax, where a unit is (sequence,
+//     KV head, group of <= 8 query heads) and pmax = ceil(max_seq_len / 16).
+//     It is cut evenly over persistent CTAs (one per SM), so every SM streams
+//     the same number of pages whatever the batch shape (stream-K style); a
+//     CTA walks its range unit by unit ("segments").
+//   * Each of the CTA's warps takes every NW-th page of that range and streams
+//     it through its own ring of shared-memory stages: the warp issues one TMA
+//     tensor copy per K/V tile (plus the NVFP4 block scales) into a stage,
+//     completion tracked by that stage's mbarrier, and refills the stage as
+//     soon as its contents are in registers.  Block ids are gathered 32 pages
+//     ahead (one coalesced load per 32 pages).  Tiles are 128/64/32-byte
+//     swizzled so the fragment reads are bank-conflict free.  A warp only
+//     waits on barriers of its own stages, one phase at a time.
 //   * The G (<= 8) query heads sharing a KV head make QK^T and PV small
 //     contractions, run on tensor cores with mma.sync m16n8k16 and fp32
 //     accumulation: S^T[16 tokens][8 heads] = K_codes . Q^T, then
@@ -31,10 +36,10 @@
 //   * P is split into a 16-bit high part and a 16-bit residual (two MMAs) so
 //     the probabilities keep ~22 bits: rounding P to one 16-bit value would
 //     cost up to 2^-11 relative on outputs whose V reaches hundreds.
-//   * Online softmax in the exp2 domain per warp; warps are merged through
-//     shared memory; splits are merged by the last CTA of each (sequence, KV
-//     head) to arrive (atomic ticket, nobody waits), which writes out and lse.
-//     With one split the CTA writes the result directly.
+//   * Online softmax in the exp2 domain per warp (rescale skipped when no
+//     running max moved).  At a segment end the consumer warps merge through
+//     shared memory; a unit split over several CTAs is merged by the last of
+//     them to arrive (atomic ticket, nobody waits), which writes out and lse.
 #include <math.h>
 
 #include "kvq_device.cuh"
@@ -47,7 +52,6 @@ namespace {
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kPScale = 4096.0f;  // P is fed to the MMA as p * 2^12 (exact)
-constexpr int kMaxSplits = 512;
 
 // --------------------------------------------------------------------------
 // Per-(format, head_dim) fragment layouts.
@@ -402,13 +406,17 @@ struct Fmt<2, 128> {
 };
 
 // Kernel shape per format: warps per CTA and stages per warp.
+// Kernel shape per format: warps per CTA (NW, one CTA per SM) and ring stages
+// per warp (NSW).  Each warp owns NSW stages (~150 KB of ring per SM in all)
+// and refills a stage only after consuming it, so every mbarrier wait is
+// exactly one phase ahead; NW warp-partial slots serve the segment merge.
 template <int FMT, int D>
 struct Shape {
-  static constexpr int NW = 4;
-  static constexpr int NS = Fmt<FMT, D>::STAGE <= 1280 ? 8
-                            : Fmt<FMT, D>::STAGE <= 2560 ? 6
-                            : Fmt<FMT, D>::STAGE <= 4096 ? 4
-                                                        : 3;
+  static constexpr int NW = (FMT == 0 && D == 128) ? 10 : 12;
+  static constexpr int STAGE = Fmt<FMT, D>::STAGE;
+  static constexpr int NSW = STAGE <= 1280 ? 10 : STAGE <= 2048 ? 6 : STAGE <= 2560 ? 5
+                             : STAGE <= 4096 ? 3 : 2;
+  static constexpr int WPART = 16 + 8 * D;  // floats of one partial: m[8], l[8], o[8][D]
 };
 
 template <bool BF>
@@ -419,10 +427,119 @@ __device__ __forceinline__ void mma16816(float c[4], const uint32_t a[4], uint32
     mma_f16(c, a, b0, b1);
 }
 
-template <int FMT, int D>
-__device__ __forceinline__ void drain(uint64_t* bars, int from, int to) {
-  constexpr int NS = Shape<FMT, D>::NS;
-  for (int k = from; k < to; ++k) mbar_wait_bounded(&bars[k % NS], (k / NS) & 1);
+// The CTA that holds virtual page g when V pages are split evenly over C CTAs
+// (CTA c owns [c*V/C, (c+1)*V/C)).
+__device__ __forceinline__ int cta_of(int64_t g, int64_t V, int C) {
+  return static_cast<int>(((g + 1) * C - 1) / V);
+}
+
+struct UnitView {
+  int b, h, grp, len;
+  int ps, pe;  // this CTA's page range of the unit, clipped to its length
+};
+
+__device__ __forceinline__ int ps_of(const DecodeParams& p, int u, int64_t vbeg) {
+  const int64_t base = static_cast<int64_t>(u) * p.pmax;
+  return vbeg > base ? static_cast<int>(vbeg - base) : 0;
+}
+
+__device__ __forceinline__ UnitView unit_view(const DecodeParams& p, int u, int64_t vbeg,
+                                              int64_t vend) {
+  UnitView v;
+  v.grp = u % p.n_groups;
+  v.h = (u / p.n_groups) % p.Hkv;
+  v.b = u / (p.n_groups * p.Hkv);
+  int len = __ldg(p.seq_lens + v.b);
+  if (len < 0 || len > p.max_seq_len) len = 0;  // reported by the unit's first CTA
+  v.len = len;
+  const int64_t base = static_cast<int64_t>(u) * p.pmax;
+  const int npages = (len + kPage - 1) / kPage;
+  v.ps = ps_of(p, u, vbeg);
+  const int pe = static_cast<int>((vend < base + p.pmax ? vend : base + p.pmax) - base);
+  v.pe = pe < npages ? pe : npages;
+  if (v.pe < v.ps) v.pe = v.ps;
+  return v;
+}
+
+// The units a CTA's range covers, built once at kernel start (one load round):
+// kend[i] = items (cached pages) of units u0..u0+i, len[i] = length of u0+i.
+constexpr int kMaxUnits = 64;
+struct UnitTable {
+  int n, total;
+  int kend[kMaxUnits];
+  int len[kMaxUnits];
+};
+
+// Block id and KV head of the CTA's item k, or blk = -1 past the last item.
+__device__ __forceinline__ void item_block(const DecodeParams& p, const UnitTable& tab, int u0,
+                                           int64_t vbeg, int64_t vend, int k, int& blk, int& h) {
+  blk = -1;
+  h = 0;
+  if (k >= tab.total) return;
+  int i = 0, k0 = 0;
+  if (tab.n <= kMaxUnits) {
+    int lo = 0, hi = tab.n - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if (tab.kend[mid] > k)
+        hi = mid;
+      else
+        lo = mid + 1;
+    }
+    i = lo;
+    k0 = i ? tab.kend[i - 1] : 0;
+  } else {  // long unit lists: walk them
+    for (;;) {
+      const UnitView uv = unit_view(p, u0 + i, vbeg, vend);
+      if (k < k0 + uv.pe - uv.ps) break;
+      k0 += uv.pe - uv.ps;
+      ++i;
+    }
+  }
+  const int u = u0 + i;
+  h = (u / p.n_groups) % p.Hkv;
+  const int b = u / (p.n_groups * p.Hkv);
+  blk = __ldg(p.block_table + static_cast<size_t>(b) * p.max_blocks + ps_of(p, u, vbeg) + (k - k0));
+}
+
+// Merge the per-CTA partials of unit u (slots u + c for c in [c_first,
+// c_first + n)) into out / lse; threads t of nthreads share the float4
+// columns.  One pass with a running maximum, so the loads of several partials
+// are in flight together.
+template <int D, int WPART>
+__device__ __forceinline__ void final_merge(const DecodeParams& p, int u, int b, int h, int grp,
+                                            int c_first, int n, float vs, int t, int nthreads) {
+  const float kInf = __int_as_float(0x7f800000);
+  const float* up = p.ws_part + (static_cast<size_t>(u) + c_first) * WPART;
+  for (int col = t; col < 2 * D; col += nthreads) {  // float4 columns of [8][D]
+    const int hh = col / (D / 4), d4 = (col - hh * (D / 4)) * 4;
+    const int qi = grp * 8 + hh;
+    if (qi >= p.G) continue;
+    float M = -kInf, L = 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+    for (int s = 0; s < n; ++s) {
+      const float* ps = up + s * WPART;
+      const float m = __ldcg(ps + hh);
+      const float l = __ldcg(ps + 8 + hh);
+      const float4 v4 = __ldcg(reinterpret_cast<const float4*>(ps + 16 + hh * D + d4));
+      if (m != -kInf) {
+        const float mn = fmaxf(M, m);
+        const float a = M == -kInf ? 0.f : fast_exp2(M - mn), e = fast_exp2(m - mn);
+        L = L * a + l * e;
+        acc.x = acc.x * a + v4.x * e;
+        acc.y = acc.y * a + v4.y * e;
+        acc.z = acc.z * a + v4.z * e;
+        acc.w = acc.w * a + v4.w * e;
+        M = mn;
+      }
+    }
+    const float sc = L > 0.f ? vs / (L * kPScale) : 0.f;
+    const size_t row = static_cast<size_t>(b) * p.Hq + h * p.G + qi;
+    *reinterpret_cast<float4*>(p.out + row * D + d4) =
+        make_float4(acc.x * sc, acc.y * sc, acc.z * sc, acc.w * sc);
+    if (d4 == 0 && p.lse) p.lse[row] = L > 0.f ? (M + log2f(L)) * kLn2 : -kInf;
+  }
 }
 
 template <int FMT, int D>
@@ -431,25 +548,38 @@ __global__ void __launch_bounds__(Shape<FMT, D>::NW * 32, 1)
                       const __grid_constant__ CUtensorMap mks,
                       const __grid_constant__ CUtensorMap mvs, const DecodeParams p) {
   using F = Fmt<FMT, D>;
-  constexpr int NW = Shape<FMT, D>::NW, NS = Shape<FMT, D>::NS;
-  constexpr int KS = D / 16, MT = D / 16;
+  using S = Shape<FMT, D>;
+  constexpr int NW = S::NW, NSW = S::NSW, KS = D / 16, MT = D / 16;
+  constexpr int NT = NW * 32;
   const float kInf = __int_as_float(0x7f800000);
 
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~static_cast<uintptr_t>(1023));
-  __shared__ int s_last;
+  uint8_t* rings = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                              ~static_cast<uintptr_t>(1023));
+  float* slots = reinterpret_cast<float*>(rings + static_cast<size_t>(NW) * NSW * F::STAGE);
+  uint64_t* bars_all = reinterpret_cast<uint64_t*>(slots + NW * S::WPART);
+  __shared__ UnitTable tab;
+  __shared__ int s_last;  // this CTA completes the unit's cross-CTA merge
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int gid = lane >> 2, tig = lane & 3;
-  uint8_t* stages = smem + static_cast<size_t>(warp) * NS * F::STAGE;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + static_cast<size_t>(NW) * NS * F::STAGE) +
-                   warp * NS;
+  const int c = blockIdx.x, C = gridDim.x;
+  const int64_t V = static_cast<int64_t>(p.units) * p.pmax;
+  uint8_t* ring = rings + static_cast<size_t>(warp) * NSW * F::STAGE;
+  uint64_t* bars = bars_all + warp * NSW;
 
-  const int split = blockIdx.x;
-  const int h = blockIdx.y / p.n_groups, grp = blockIdx.y % p.n_groups;
-  const int b = blockIdx.z;
-  const int unit = (b * p.Hkv + h) * p.n_groups + grp;
+  if (V == 0) {  // nothing cached anywhere: every output is empty
+    for (int64_t i = static_cast<int64_t>(c) * blockDim.x + tid;
+         i < static_cast<int64_t>(p.B) * p.Hq * D; i += static_cast<int64_t>(C) * blockDim.x) {
+      p.out[i] = 0.f;
+      if (p.lse && i % D == 0) p.lse[i / D] = -kInf;
+    }
+    return;
+  }
+  const int64_t vbeg = static_cast<int64_t>(c) * V / C, vend = static_cast<int64_t>(c + 1) * V / C;
+  if (vbeg >= vend) return;
+  const int u0 = static_cast<int>(vbeg / p.pmax), u1 = static_cast<int>((vend - 1) / p.pmax);
+  const int nu = u1 - u0 + 1;
 
   // Scales: FP8 needs s > 0, NVFP4 g >= 0 (0 = an all-zero tensor); both finite.
   float ks = 1.f, vs = 1.f;
@@ -461,309 +591,326 @@ __global__ void __launch_bounds__(Shape<FMT, D>::NW * 32, 1)
       scale_ok = ks > 0.f && vs > 0.f && ks < kInf && vs < kInf;
     else
       scale_ok = ks >= 0.f && vs >= 0.f && ks < kInf && vs < kInf;
-  }
-  int len = __ldg(p.seq_lens + b);
-  if (len < 0 || len > p.max_seq_len) {
-    if (tid == 0 && split == 0 && grp == 0) set_err(p.d_err, kErrSeqLen);
-    len = 0;
-  }
-  if (!scale_ok) {
-    if (tid == 0 && split == 0 && blockIdx.y == 0 && b == 0) set_err(p.d_err, kErrScale);
-    len = 0;
+    if (!scale_ok && c == 0 && tid == 0) set_err(p.d_err, kErrScale);
   }
 
-  const int n_pages = (len + kPage - 1) / kPage;
-  const int pg0 = split * p.pages_per_split;
-  const int pg1 = min(pg0 + p.pages_per_split, n_pages);
-  const int first = pg0 + warp;
-  const int n_my = first < pg1 ? (pg1 - first + NW - 1) / NW : 0;
-  const int32_t* bt = p.block_table + static_cast<size_t>(b) * p.max_blocks;
-
-  if (lane == 0) {
-#pragma unroll
-    for (int i = 0; i < NS; ++i) mbar_init(&bars[i], 1);
-    mbar_init_fence();
-  }
-  __syncwarp();
-
-  // Issue the copies of this warp's i-th page into stage i % NS (lane 0).
-  auto issue = [&](int i) {
-    const int blk = __ldg(bt + first + i * NW);
-    uint64_t* bar = &bars[i % NS];
-    if (blk >= 0 && blk < p.num_blocks) {
-      F::issue(stages + (i % NS) * F::STAGE, bar, &mk, &mv, &mks, &mvs, h, blk);
-    } else {
-      set_err(p.d_err, kErrBlockId);
-      mbar_arrive(bar);  // completes the phase with no data; the page is skipped
-    }
-  };
-  if (lane == 0) {
-    const int n0 = n_my < NS ? n_my : NS;
-    for (int i = 0; i < n0; ++i) issue(i);
-  }
-
-  // Query fragments (B operand of QK), head gid of this group; padded heads 0.
-  const float c_log2 = p.sm_scale * ks * kLog2e;
+  // Query fragments (B operand of QK) of unit u; padded heads are 0.  The
+  // thread's head-dim elements come in 16-byte runs of 8.
   uint32_t qb[KS][2];
-  {
+  auto load_q = [&](int u) {
+    const int grp = u % p.n_groups, h = (u / p.n_groups) % p.Hkv, b = u / (p.n_groups * p.Hkv);
     const int qi = grp * 8 + gid;
     const bool hv = qi < p.G;
     const uint16_t* qrow = p.q + (static_cast<size_t>(b) * p.Hq + h * p.G + (hv ? qi : 0)) * D;
 #pragma unroll
-    for (int s = 0; s < KS; ++s) {
+    for (int i = 0; i < D / 4; i += 8) {
+      const uint4 w = hv ? __ldg(reinterpret_cast<const uint4*>(qrow + F::k_elem(tig, i)))
+                         : make_uint4(0u, 0u, 0u, 0u);
+      const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        const int e0 = F::k_elem(tig, 4 * s + 2 * half);
-        const uint32_t a = hv ? __ldg(qrow + e0) : 0u;
-        const uint32_t c = hv ? __ldg(qrow + e0 + 1) : 0u;
-        if constexpr (F::kBF16)
-          qb[s][half] = a | (c << 16);
-        else
-          qb[s][half] = pack_f16x2(__uint_as_float(a << 16), __uint_as_float(c << 16));
+      for (int x = 0; x < 4; ++x) {
+        uint32_t v = ws[x];
+        if constexpr (!F::kBF16) v = pack_f16x2(bf16_lo(v), bf16_hi(v));
+        qb[i / 4 + x / 2][x & 1] = v;
       }
+    }
+  };
+  load_q(u0);  // in flight while the unit table is built
+
+  // ---- unit table: lane i of warp 0 looks at unit u0 + i (32 at a time)
+  if (warp == 0) {
+    int run = 0;
+    for (int base = 0; base < nu; base += 32) {
+      const int i = base + lane;
+      int n_i = 0, len_i = 0;
+      if (i < nu) {
+        const UnitView uv = unit_view(p, u0 + i, vbeg, vend);
+        n_i = scale_ok ? uv.pe - uv.ps : 0;
+        len_i = uv.len;
+      }
+      int x = n_i;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, off);
+        if (lane >= off) x += y;
+      }
+      if (i < nu && i < kMaxUnits) {
+        tab.kend[i] = run + x;
+        tab.len[i] = len_i;
+      }
+      run += __shfl_sync(0xffffffffu, x, 31);
+    }
+    if (lane == 0) {
+      tab.n = nu;
+      tab.total = run;
+#pragma unroll 1
+      for (int i = 0; i < NW * NSW; ++i) mbar_init(&bars_all[i], 1);
+      mbar_init_fence();
     }
   }
+  __syncthreads();
+  const int total = tab.total;
+  const int n_local = warp < total ? (total - warp + NW - 1) / NW : 0;
 
-  float m0 = -kInf, m1 = -kInf, l0 = 0.f, l1 = 0.f;
-  float o[MT][4];
-#pragma unroll
-  for (int j = 0; j < MT; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
+  // Block ids of this warp's local items [chunk, chunk + 64): lane L holds
+  // items chunk + L (cur) and chunk + 32 + L (nxt).
+  int chunk = 0;
+  int cur_blk, cur_h, nxt_blk, nxt_h;
+  item_block(p, tab, u0, vbeg, vend, warp + lane * NW, cur_blk, cur_h);
+  item_block(p, tab, u0, vbeg, vend, warp + (32 + lane) * NW, nxt_blk, nxt_h);
 
-  for (int i = 0; i < n_my; ++i) {
-    const int st = i % NS;
-    const int page = first + i * NW;
-    const int blk = __ldg(bt + page);
-    // all lanes agree on the outcome so the warp stays converged
-    if (!__all_sync(0xffffffffu, mbar_wait_bounded(&bars[st], (i / NS) & 1))) {
-      if (lane == 0) set_err(p.d_err, kErrTimeout);
-      drain<FMT, D>(bars, i + 1, min(i + NS, n_my));
-      break;
+  // Issue the copies of local item i into stage i % NSW (all lanes call;
+  // lane 0 issues).  stage_ok (warp-uniform) records which stages hold a
+  // valid page; a bad block id completes its stage's phase with no data.
+  unsigned stage_ok = 0;
+  auto issue = [&](int i) {
+    if (i >= chunk + 32) {  // slide the id window by 32 items
+      chunk += 32;
+      cur_blk = nxt_blk;
+      cur_h = nxt_h;
+      item_block(p, tab, u0, vbeg, vend, warp + (chunk + 32 + lane) * NW, nxt_blk, nxt_h);
     }
-    if (blk < 0 || blk >= p.num_blocks) {  // reported at issue time; skip
-      __syncwarp();
-      if (lane == 0 && i + NS < n_my) issue(i + NS);
-      continue;
-    }
-    const uint8_t* sp = stages + st * F::STAGE;
-    const int n_valid = min(kPage, len - page * kPage);
-
-    // ---- S^T = K Q^T on tensor cores (two accumulator chains)
-    uint32_t ka[KS][4];
-    F::load_k(sp, gid, tig, ka);
-    float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-    for (int s = 0; s < KS; ++s) {
-      if (s & 1)
-        mma16816<F::kBF16>(sb, ka[s], qb[s][0], qb[s][1]);
-      else
-        mma16816<F::kBF16>(sa, ka[s], qb[s][0], qb[s][1]);
-    }
-    uint32_t va[MT][4];
-    F::load_v(sp, gid, tig, va);
-
-    // The stage is now in registers: hand it back to TMA for page i + NS.
-    __syncwarp();
-    if (lane == 0 && i + NS < n_my) {
-      fence_proxy_async_smem();
-      issue(i + NS);
-    }
-
-    float s0 = (sa[0] + sb[0]) * c_log2, s1 = (sa[1] + sb[1]) * c_log2;
-    float s2 = (sa[2] + sb[2]) * c_log2, s3 = (sa[3] + sb[3]) * c_log2;
-    if (n_valid < kPage) {  // last, partial page: mask tokens past the length
-      if (gid >= n_valid) s0 = s1 = -kInf;
-      if (gid + 8 >= n_valid) s2 = s3 = -kInf;
-      const uint32_t m01 = (2 * tig < n_valid ? 0x0000FFFFu : 0u) |
-                           (2 * tig + 1 < n_valid ? 0xFFFF0000u : 0u);
-      const uint32_t m23 = (2 * tig + 8 < n_valid ? 0x0000FFFFu : 0u) |
-                           (2 * tig + 9 < n_valid ? 0xFFFF0000u : 0u);
-#pragma unroll
-      for (int j = 0; j < MT; ++j) {  // unwritten slots may hold NaN codes
-        va[j][0] &= m01;
-        va[j][1] &= m01;
-        va[j][2] &= m23;
-        va[j][3] &= m23;
+    const int blk = __shfl_sync(0xffffffffu, cur_blk, i - chunk);
+    const int h = __shfl_sync(0xffffffffu, cur_h, i - chunk);
+    const bool ok = blk >= 0 && blk < p.num_blocks;
+    stage_ok = (stage_ok & ~(1u << (i % NSW))) | (static_cast<unsigned>(ok) << (i % NSW));
+    if (lane == 0) {
+      uint64_t* bar = &bars[i % NSW];
+      if (ok) {
+        F::issue(ring + (i % NSW) * F::STAGE, bar, &mk, &mv, &mks, &mvs, h, blk);
+      } else {
+        set_err(p.d_err, kErrBlockId);
+        mbar_arrive(bar);  // completes the phase with no data; the page is skipped
       }
     }
+  };
+  for (int i = 0; i < NSW && i < n_local; ++i) issue(i);
 
-    // ---- online softmax (log2 domain); this thread: heads 2tig, 2tig+1
-    float mx0 = fmaxf(s0, s2), mx1 = fmaxf(s1, s3);
+  const float c_log2 = p.sm_scale * ks * kLog2e;
+  int k_base = 0, j = 0;  // j = this warp's next local item
+  for (int si = 0; si < nu; ++si) {
+    const int u = u0 + si;
+    const int grp = u % p.n_groups, h = (u / p.n_groups) % p.Hkv, b = u / (p.n_groups * p.Hkv);
+    int n_items, len;
+    if (nu <= kMaxUnits) {
+      n_items = tab.kend[si] - (si ? tab.kend[si - 1] : 0);
+      len = tab.len[si];
+    } else {
+      const UnitView uv = unit_view(p, u, vbeg, vend);
+      n_items = scale_ok ? uv.pe - uv.ps : 0;
+      len = uv.len;
+    }
+    const int ps = ps_of(p, u, vbeg);
+    const int c_first = cta_of(static_cast<int64_t>(u) * p.pmax, V, C);
+    const int c_last = cta_of(static_cast<int64_t>(u + 1) * p.pmax - 1, V, C);
+    if (c == c_first && tid == 0 && h == 0 && grp == 0) {
+      const int raw = __ldg(p.seq_lens + b);
+      if (raw < 0 || raw > p.max_seq_len) set_err(p.d_err, kErrSeqLen);
+    }
+    if (si > 0) load_q(u);
+
+    float m0 = -kInf, m1 = -kInf, l0 = 0.f, l1 = 0.f;
+    float o[MT][4];
+#pragma unroll
+    for (int jj = 0; jj < MT; ++jj) o[jj][0] = o[jj][1] = o[jj][2] = o[jj][3] = 0.f;
+
+    const int k_end = k_base + n_items;
+    for (int k = warp + j * NW; k < k_end; k += NW, ++j) {
+      const int st = j % NSW;
+      const uint8_t* sp = ring + st * F::STAGE;
+      // all lanes agree on the outcome so the warp stays converged
+      if (!__all_sync(0xffffffffu, mbar_wait_bounded(&bars[st], (j / NSW) & 1))) {
+        if (lane == 0) set_err(p.d_err, kErrTimeout);
+        for (int i = j + 1; i < j + NSW && i < n_local; ++i)  // drain copies in flight
+          mbar_wait_bounded(&bars[i % NSW], (i / NSW) & 1);
+        j = n_local;
+        break;
+      }
+      const int page = ps + (k - k_base);
+      const int n_valid = min(kPage, len - page * kPage);
+      const bool valid = (stage_ok >> st) & 1u;
+
+      uint32_t ka[KS][4], va[MT][4];
+      float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
+      if (valid) {
+        // ---- S^T = K Q^T on tensor cores (two accumulator chains)
+        F::load_k(sp, gid, tig, ka);
+#pragma unroll
+        for (int s = 0; s < KS; ++s) {
+          if (s & 1)
+            mma16816<F::kBF16>(sb, ka[s], qb[s][0], qb[s][1]);
+          else
+            mma16816<F::kBF16>(sa, ka[s], qb[s][0], qb[s][1]);
+        }
+        F::load_v(sp, gid, tig, va);
+      }
+      // the stage is in registers: refill it with local item j + NSW
+      __syncwarp();
+      if (j + NSW < n_local) {
+        if (lane == 0) fence_proxy_async_smem();
+        issue(j + NSW);
+      }
+      if (!valid) continue;
+
+      float s0 = (sa[0] + sb[0]) * c_log2, s1 = (sa[1] + sb[1]) * c_log2;
+      float s2 = (sa[2] + sb[2]) * c_log2, s3 = (sa[3] + sb[3]) * c_log2;
+      if (n_valid < kPage) {  // last, partial page: mask tokens past the length
+        if (gid >= n_valid) s0 = s1 = -kInf;
+        if (gid + 8 >= n_valid) s2 = s3 = -kInf;
+        const uint32_t m01 = (2 * tig < n_valid ? 0x0000FFFFu : 0u) |
+                             (2 * tig + 1 < n_valid ? 0xFFFF0000u : 0u);
+        const uint32_t m23 = (2 * tig + 8 < n_valid ? 0x0000FFFFu : 0u) |
+                             (2 * tig + 9 < n_valid ? 0xFFFF0000u : 0u);
+#pragma unroll
+        for (int jj = 0; jj < MT; ++jj) {  // unwritten slots may hold NaN codes
+          va[jj][0] &= m01;
+          va[jj][1] &= m01;
+          va[jj][2] &= m23;
+          va[jj][3] &= m23;
+        }
+      }
+
+      // ---- online softmax (log2 domain); this thread: heads 2tig, 2tig+1
+      float mx0 = fmaxf(s0, s2), mx1 = fmaxf(s1, s3);
+#pragma unroll
+      for (int off = 4; off < 32; off <<= 1) {
+        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+      }
+      const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
+      if (__any_sync(0xffffffffu, mn0 != m0 || mn1 != m1)) {
+        const float a0 = fast_exp2(m0 - mn0), a1 = fast_exp2(m1 - mn1);
+        l0 *= a0;
+        l1 *= a1;
+#pragma unroll
+        for (int jj = 0; jj < MT; ++jj) {
+          o[jj][0] *= a0;
+          o[jj][1] *= a1;
+          o[jj][2] *= a0;
+          o[jj][3] *= a1;
+        }
+        m0 = mn0;
+        m1 = mn1;
+      }
+      const float p0 = fast_exp2(s0 - m0), p1 = fast_exp2(s1 - m1);
+      const float p2 = fast_exp2(s2 - m0), p3 = fast_exp2(s3 - m1);
+      l0 += p0 + p2;
+      l1 += p1 + p3;
+
+      // ---- P^T fragments: high part + residual, transposed in registers
+      const float q0 = p0 * kPScale, q1 = p1 * kPScale, q2 = p2 * kPScale, q3 = p3 * kPScale;
+      uint32_t x0h, x1h, x0l, x1l;
+      float r0, r1, r2, r3;
+      if constexpr (F::kBF16) {
+        x0h = pack_bf16x2(q0, q1);
+        x1h = pack_bf16x2(q2, q3);
+        unpack_bf16x2(x0h, r0, r1);
+        unpack_bf16x2(x1h, r2, r3);
+        x0l = pack_bf16x2(q0 - r0, q1 - r1);
+        x1l = pack_bf16x2(q2 - r2, q3 - r3);
+      } else {
+        x0h = pack_f16x2(q0, q1);
+        x1h = pack_f16x2(q2, q3);
+        unpack_f16x2(x0h, r0, r1);
+        unpack_f16x2(x1h, r2, r3);
+        x0l = pack_f16x2(q0 - r0, q1 - r1);
+        x1l = pack_f16x2(q2 - r2, q3 - r3);
+      }
+      const uint32_t bh0 = movmatrix_t(x0h), bh1 = movmatrix_t(x1h);
+      const uint32_t bl0 = movmatrix_t(x0l), bl1 = movmatrix_t(x1l);
+
+      // ---- O^T += V^T P^T
+#pragma unroll
+      for (int jj = 0; jj < MT; ++jj) {
+        mma16816<F::kBF16>(o[jj], va[jj], bh0, bh1);
+        mma16816<F::kBF16>(o[jj], va[jj], bl0, bl1);
+      }
+    }
+    k_base = k_end;
+
 #pragma unroll
     for (int off = 4; off < 32; off <<= 1) {
-      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
-      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+      l0 += __shfl_xor_sync(0xffffffffu, l0, off);
+      l1 += __shfl_xor_sync(0xffffffffu, l1, off);
     }
-    const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
-    const float a0 = fast_exp2(m0 - mn0), a1 = fast_exp2(m1 - mn1);
-    m0 = mn0;
-    m1 = mn1;
-    const float p0 = fast_exp2(s0 - mn0), p1 = fast_exp2(s1 - mn1);
-    const float p2 = fast_exp2(s2 - mn0), p3 = fast_exp2(s3 - mn1);
-    l0 = l0 * a0 + (p0 + p2);
-    l1 = l1 * a1 + (p1 + p3);
-#pragma unroll
-    for (int j = 0; j < MT; ++j) {
-      o[j][0] *= a0;
-      o[j][1] *= a1;
-      o[j][2] *= a0;
-      o[j][3] *= a1;
+    // ---- segment end: warp partials -> shared slots, merged by the CTA
+    float* wp = slots + warp * S::WPART;  // m[8], l[8], o[8][D]
+    if (gid == 0) {
+      wp[2 * tig] = m0;
+      wp[2 * tig + 1] = m1;
+      wp[8 + 2 * tig] = l0;
+      wp[8 + 2 * tig + 1] = l1;
     }
-
-    // ---- P^T fragments: high part + residual, transposed in registers
-    const float q0 = p0 * kPScale, q1 = p1 * kPScale, q2 = p2 * kPScale, q3 = p3 * kPScale;
-    uint32_t x0h, x1h, x0l, x1l;
-    float r0, r1, r2, r3;
-    if constexpr (F::kBF16) {
-      x0h = pack_bf16x2(q0, q1);
-      x1h = pack_bf16x2(q2, q3);
-      unpack_bf16x2(x0h, r0, r1);
-      unpack_bf16x2(x1h, r2, r3);
-      x0l = pack_bf16x2(q0 - r0, q1 - r1);
-      x1l = pack_bf16x2(q2 - r2, q3 - r3);
-    } else {
-      x0h = pack_f16x2(q0, q1);
-      x1h = pack_f16x2(q2, q3);
-      unpack_f16x2(x0h, r0, r1);
-      unpack_f16x2(x1h, r2, r3);
-      x0l = pack_f16x2(q0 - r0, q1 - r1);
-      x1l = pack_f16x2(q2 - r2, q3 - r3);
+#pragma unroll
+    for (int jj = 0; jj < MT; ++jj) {
+      const int d0 = F::v_elem(gid, 2 * jj), d1 = F::v_elem(gid, 2 * jj + 1);
+      wp[16 + (2 * tig) * D + d0] = o[jj][0];
+      wp[16 + (2 * tig + 1) * D + d0] = o[jj][1];
+      wp[16 + (2 * tig) * D + d1] = o[jj][2];
+      wp[16 + (2 * tig + 1) * D + d1] = o[jj][3];
     }
-    const uint32_t bh0 = movmatrix_t(x0h), bh1 = movmatrix_t(x1h);
-    const uint32_t bl0 = movmatrix_t(x0l), bl1 = movmatrix_t(x1l);
-
-    // ---- O^T += V^T P^T
+    __syncthreads();
+    const bool alone = c_first == c_last;
+    float* gpart = p.ws_part + (static_cast<size_t>(u) + c) * S::WPART;
+    for (int idx = tid; idx < 8 * D; idx += NT) {
+      const int hh = idx / D, d = idx - hh * D;
+      float M = -kInf;
 #pragma unroll
-    for (int j = 0; j < MT; ++j) {
-      mma16816<F::kBF16>(o[j], va[j], bh0, bh1);
-      mma16816<F::kBF16>(o[j], va[j], bl0, bl1);
-    }
-  }
-
-  // ---- warp partial -> shared memory (this warp's own, now idle, stages)
+      for (int w = 0; w < NW; ++w) M = fmaxf(M, slots[w * S::WPART + hh]);
+      float L = 0.f, acc = 0.f;
+      if (M != -kInf) {
 #pragma unroll
-  for (int off = 4; off < 32; off <<= 1) {
-    l0 += __shfl_xor_sync(0xffffffffu, l0, off);
-    l1 += __shfl_xor_sync(0xffffffffu, l1, off);
-  }
-  __syncwarp();
-  float* wml = reinterpret_cast<float*>(stages);  // m[8], l[8], o[8][D]
-  if (gid == 0) {
-    wml[2 * tig] = m0;
-    wml[2 * tig + 1] = m1;
-    wml[8 + 2 * tig] = l0;
-    wml[8 + 2 * tig + 1] = l1;
-  }
-  float* wo = wml + 16;
-#pragma unroll
-  for (int j = 0; j < MT; ++j) {
-    const int d0 = F::v_elem(gid, 2 * j), d1 = F::v_elem(gid, 2 * j + 1);
-    wo[(2 * tig) * D + d0] = o[j][0];
-    wo[(2 * tig + 1) * D + d0] = o[j][1];
-    wo[(2 * tig) * D + d1] = o[j][2];
-    wo[(2 * tig + 1) * D + d1] = o[j][3];
-  }
-  __syncthreads();
-
-  // ---- merge the warps: (M, L, O) of the CTA for each of the 8 heads
-  constexpr int WSTRIDE = NS * F::STAGE / 4;  // floats between warp partials
-  const float* base = reinterpret_cast<const float*>(smem);
-  for (int idx = tid; idx < 8 * D; idx += NW * 32) {
-    const int hh = idx / D, d = idx - hh * D;
-    float M = -kInf;
-#pragma unroll
-    for (int w = 0; w < NW; ++w) M = fmaxf(M, base[w * WSTRIDE + hh]);
-    float L = 0.f, acc = 0.f;
-    if (M != -kInf) {
-#pragma unroll
-      for (int w = 0; w < NW; ++w) {
-        const float e = fast_exp2(base[w * WSTRIDE + hh] - M);
-        L += e * base[w * WSTRIDE + 8 + hh];
-        acc += e * base[w * WSTRIDE + 16 + hh * D + d];
+        for (int w = 0; w < NW; ++w) {
+          const float e = fast_exp2(slots[w * S::WPART + hh] - M);
+          L += e * slots[w * S::WPART + 8 + hh];
+          acc += e * slots[w * S::WPART + 16 + hh * D + d];
+        }
+      }
+      if (alone) {
+        const int qi = grp * 8 + hh;
+        if (qi < p.G) {
+          const size_t row = static_cast<size_t>(b) * p.Hq + h * p.G + qi;
+          p.out[row * D + d] = L > 0.f ? acc * (vs / (L * kPScale)) : 0.f;
+          if (d == 0 && p.lse) p.lse[row] = L > 0.f ? (M + log2f(L)) * kLn2 : -kInf;
+        }
+      } else {
+        gpart[16 + hh * D + d] = acc;
+        if (d == 0) {
+          gpart[hh] = M;
+          gpart[8 + hh] = L;
+        }
       }
     }
-    if (p.num_splits == 1) {
-      const int qi = grp * 8 + hh;
-      if (qi < p.G) {
-        const size_t row = static_cast<size_t>(b) * p.Hq + h * p.G + qi;
-        p.out[row * D + d] = L > 0.f ? acc * (vs / (L * kPScale)) : 0.f;
-        if (d == 0 && p.lse) p.lse[row] = L > 0.f ? (M + log2f(L)) * kLn2 : -kInf;
+    if (!alone) {
+      // ---- the last CTA of the unit to get here merges all its partials
+      __threadfence();
+      __syncthreads();
+      if (tid == 0) {
+        const unsigned t = atomicAdd(p.ws_cnt + u, 1u);
+        s_last = (t == static_cast<unsigned>(c_last - c_first));
       }
-    } else {
-      const size_t pi = (static_cast<size_t>(unit) * p.num_splits + split) * 8 + hh;
-      p.ws_o[pi * D + d] = acc;
-      if (d == 0) {
-        p.ws_ml[pi * 2] = M;
-        p.ws_ml[pi * 2 + 1] = L;
+      __syncthreads();
+      if (s_last) {
+        __threadfence();
+        final_merge<D, S::WPART>(p, u, b, h, grp, c_first, c_last - c_first + 1, vs, tid, NT);
+        if (tid == 0) p.ws_cnt[u] = 0u;  // ready for the next launch
       }
     }
+    __syncthreads();  // slots and s_last are reused by the next segment
   }
-  if (p.num_splits == 1) return;
-
-  // ---- split-K merge by the last CTA of this (sequence, KV head, group)
-  __threadfence();
-  __syncthreads();
-  if (tid == 0) {
-    const unsigned t = atomicAdd(p.ws_cnt + unit, 1u);
-    s_last = (t == static_cast<unsigned>(p.num_splits - 1));
-  }
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
-
-  const int S = p.num_splits;
-  const size_t ubase = static_cast<size_t>(unit) * S * 8;
-  float* wgt = reinterpret_cast<float*>(smem);  // [8][S] weights, then M[8], L[8]
-  float* hM = wgt + 8 * kMaxSplits;
-  float* hL = hM + 8;
-  // per head: M = max_s m_s, L = sum_s 2^(m_s - M) l_s (one warp per head)
-  for (int hh = warp; hh < 8; hh += NW) {
-    float M = -kInf;
-    for (int s = lane; s < S; s += 32) M = fmaxf(M, __ldcg(p.ws_ml + (ubase + s * 8 + hh) * 2));
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-    float L = 0.f;
-    for (int s = lane; s < S; s += 32) {
-      const float ms = __ldcg(p.ws_ml + (ubase + s * 8 + hh) * 2);
-      const float e = M != -kInf ? fast_exp2(ms - M) : 0.f;
-      wgt[hh * kMaxSplits + s] = e;
-      L += e * __ldcg(p.ws_ml + (ubase + s * 8 + hh) * 2 + 1);
-    }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
-    if (lane == 0) {
-      hM[hh] = M;
-      hL[hh] = L;
-    }
-  }
-  __syncthreads();
-  for (int idx = tid; idx < 8 * D; idx += NW * 32) {
-    const int hh = idx / D, d = idx - hh * D;
-    const int qi = grp * 8 + hh;
-    if (qi >= p.G) continue;
-    float acc = 0.f;
-    for (int s = 0; s < S; ++s)
-      acc += wgt[hh * kMaxSplits + s] * __ldcg(p.ws_o + (ubase + s * 8 + hh) * D + d);
-    const float L = hL[hh];
-    const size_t row = static_cast<size_t>(b) * p.Hq + h * p.G + qi;
-    p.out[row * D + d] = L > 0.f ? acc * (vs / (L * kPScale)) : 0.f;
-    if (d == 0 && p.lse) p.lse[row] = L > 0.f ? (hM[hh] + log2f(L)) * kLn2 : -kInf;
-  }
-  if (tid == 0) p.ws_cnt[unit] = 0u;  // leave the counter ready for the next launch
 }
 
 template <int FMT, int D>
 size_t smem_bytes() {
-  using F = Fmt<FMT, D>;
-  constexpr int NW = Shape<FMT, D>::NW, NS = Shape<FMT, D>::NS;
-  size_t stages = static_cast<size_t>(NW) * NS * F::STAGE;
-  size_t merge = (8 * kMaxSplits + 16) * sizeof(float);
-  size_t body = stages > merge ? stages : merge;
-  return 1024 + body + static_cast<size_t>(NW) * NS * 8;
+  using S = Shape<FMT, D>;
+  return 1024 + static_cast<size_t>(S::NW) * S::NSW * S::STAGE +
+         sizeof(float) * S::NW * S::WPART + 8 * static_cast<size_t>(S::NW) * S::NSW;
 }
 
 template <int FMT, int D>
-cudaError_t launch_t(const CUtensorMap* maps, const DecodeParams& p, cudaStream_t stream) {
-  constexpr int NW = Shape<FMT, D>::NW;
+cudaError_t launch_t(const CUtensorMap* maps, const DecodeParams& p, int ctas,
+                     cudaStream_t stream) {
+  using S = Shape<FMT, D>;
   const size_t smem = smem_bytes<FMT, D>();
   static bool attr_set = false;
   if (!attr_set) {
@@ -773,36 +920,23 @@ cudaError_t launch_t(const CUtensorMap* maps, const DecodeParams& p, cudaStream_
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  dim3 grid(p.num_splits, p.Hkv * p.n_groups, p.B);
-  kvq_decode_kernel<FMT, D><<<grid, NW * 32, smem, stream>>>(maps[0], maps[1], maps[2], maps[3], p);
+  kvq_decode_kernel<FMT, D><<<ctas, S::NW * 32, smem, stream>>>(maps[0], maps[1], maps[2],
+                                                               maps[3], p);
   return cudaGetLastError();
-}
-
-template <int FMT, int D>
-int occupancy_t() {
-  constexpr int NW = Shape<FMT, D>::NW;
-  const size_t smem = smem_bytes<FMT, D>();
-  cudaFuncSetAttribute(kvq_decode_kernel<FMT, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                       static_cast<int>(smem));
-  int n = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kvq_decode_kernel<FMT, D>, NW * 32, smem) !=
-      cudaSuccess)
-    return 0;
-  return n;
 }
 
 template <int FMT, int D>
 void config_t(DecodeConfig* c) {
   c->warps = Shape<FMT, D>::NW;
-  c->stages = Shape<FMT, D>::NS;
+  c->stages = Shape<FMT, D>::NSW;
   c->stage_bytes = Fmt<FMT, D>::STAGE;
   c->smem_bytes = smem_bytes<FMT, D>();
+  c->part_floats = Shape<FMT, D>::WPART;
 }
 
 }  // namespace
 
 bool decode_config(int fmt, int D, DecodeConfig* cfg) {
-  if (D != 64 && D != 128) return false;
   switch (fmt * 1000 + D) {
     case 64: config_t<0, 64>(cfg); return true;
     case 128: config_t<0, 128>(cfg); return true;
@@ -814,33 +948,15 @@ bool decode_config(int fmt, int D, DecodeConfig* cfg) {
   return false;
 }
 
-int decode_ctas_per_sm(int fmt, int D) {
-  static int cache[3][2] = {{-1, -1}, {-1, -1}, {-1, -1}};
-  const int di = D == 64 ? 0 : 1;
-  if (fmt < 0 || fmt > 2) return 0;
-  if (cache[fmt][di] >= 0) return cache[fmt][di];
-  int n = 0;
-  switch (fmt * 1000 + D) {
-    case 64: n = occupancy_t<0, 64>(); break;
-    case 128: n = occupancy_t<0, 128>(); break;
-    case 1064: n = occupancy_t<1, 64>(); break;
-    case 1128: n = occupancy_t<1, 128>(); break;
-    case 2064: n = occupancy_t<2, 64>(); break;
-    case 2128: n = occupancy_t<2, 128>(); break;
-  }
-  cache[fmt][di] = n;
-  return n;
-}
-
 cudaError_t launch_decode(int fmt, int D, const CUtensorMap* maps, const DecodeParams& p,
-                          cudaStream_t stream) {
+                          int ctas, cudaStream_t stream) {
   switch (fmt * 1000 + D) {
-    case 64: return launch_t<0, 64>(maps, p, stream);
-    case 128: return launch_t<0, 128>(maps, p, stream);
-    case 1064: return launch_t<1, 64>(maps, p, stream);
-    case 1128: return launch_t<1, 128>(maps, p, stream);
-    case 2064: return launch_t<2, 64>(maps, p, stream);
-    case 2128: return launch_t<2, 128>(maps, p, stream);
+    case 64: return launch_t<0, 64>(maps, p, ctas, stream);
+    case 128: return launch_t<0, 128>(maps, p, ctas, stream);
+    case 1064: return launch_t<1, 64>(maps, p, ctas, stream);
+    case 1128: return launch_t<1, 128>(maps, p, ctas, stream);
+    case 2064: return launch_t<2, 64>(maps, p, ctas, stream);
+    case 2128: return launch_t<2, 128>(maps, p, ctas, stream);
   }
   return cudaErrorInvalidValue;
 }

@@ -17,32 +17,31 @@ struct DecodeParams {
   const float* v_scale;
   float* out;                 // [B][Hq][D]
   float* lse;                 // [B][Hq] or null
-  float* ws_o;                // [units][splits][8][D]
-  float* ws_ml;               // [units][splits][8][2]
-  unsigned* ws_cnt;           // [units]
+  float* ws_part;             // [units + ctas][16 + 8 D] per-CTA partials (slot u + cta)
+  unsigned* ws_cnt;           // [units] arrival counters (zero between launches)
   int* d_err;
   int64_t num_blocks;
   int max_blocks;
   int B, Hq, Hkv, G, n_groups;
+  int units;                  // B * Hkv * n_groups (sequence, KV head, group of 8 q heads)
+  int pmax;                   // pages per unit in the work partition: ceil(max_seq_len / 16)
   int max_seq_len;
-  int num_splits, pages_per_split;
   float sm_scale;
 };
 
 struct DecodeConfig {
-  int warps;        // warps per CTA
-  int stages;       // shared-memory stages per warp
+  int warps;        // consumer warps per CTA (plus one producer warp)
+  int stages;       // shared-memory ring stages per CTA
   int stage_bytes;  // bytes per stage
   size_t smem_bytes;
+  int part_floats;  // floats of one (m, l, o) partial for 8 heads
 };
 
 // Per-(format, head_dim) kernel configuration; false if unsupported.
 bool decode_config(int fmt, int D, DecodeConfig* cfg);
-// Resident CTAs per SM of the decode kernel (occupancy), 0 on error.
-int decode_ctas_per_sm(int fmt, int D);
-// Launch the decode kernel on a (splits, Hkv*n_groups, B) grid.
+// Launch the decode kernel on `ctas` persistent CTAs.
 cudaError_t launch_decode(int fmt, int D, const CUtensorMap* maps, const DecodeParams& p,
-                          cudaStream_t stream);
+                          int ctas, cudaStream_t stream);
 
 struct QuantParams {
   const uint16_t* k;

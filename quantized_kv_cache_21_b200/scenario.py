@@ -1,0 +1,121 @@
+"""Device-resident decode workloads driven through the library's binding.
+
+A ``DecodeScenario`` builds one layer's paged cache for a named workload
+(seeded synthetic K/V, random block table, calibrated scales), then exposes the
+per-step work of a decode step: quantize-on-write of the step's new tokens
+(``write_chunk`` per sequence, through the block table) followed by the fused
+decode attention over the whole context.  Everything runs in libkvq kernels;
+torch only allocates memory and provides the stream and the RNG.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import quantized_kv_cache_21_b200 as kvq
+from quantized_kv_cache_21_b200 import workloads as wl
+
+BYTES_PER_ELEM = {"bf16": 2.0, "fp8": 1.0, "nvfp4": 4.5 / 8}
+
+
+def kv_scan_bytes(fmt: str, lens, H: int, D: int) -> int:
+    """Algorithmic bytes one decode step must read from the cache: every
+    cached token's K and V for every KV head (NVFP4 block scales included)."""
+    return int(round(sum(int(n) for n in lens) * H * 2 * D * BYTES_PER_ELEM[fmt]))
+
+
+class DecodeScenario:
+    def __init__(self, w: wl.Workload, fmt: str | None = None, device: str = "cuda",
+                 seq_offset: int = 0):
+        self.w = w
+        self.fmt = fmt or w.fmt
+        self.device = device
+        B, H, Hq, D, L = w.B, w.Hkv, w.Hq, w.D, w.seq_len
+        self.B, self.H, self.Hq, self.D, self.L = B, H, Hq, D, L
+        self.chunk = max(1, w.write_chunk)
+        self.mb = -(-L // wl.PAGE)
+        self.num_blocks = B * self.mb
+        rng = wl.rng_for(w.seed, 1)
+        self.bt = (wl.permuted_block_table(rng, B, self.mb) if w.permuted
+                   else wl.identity_block_table(B, self.mb))
+        self.lens = np.full(B, L, np.int32)
+        self.out_k = wl.outliers_for(w, H, D, "k")
+        self.out_v = wl.outliers_for(w, H, D, "v")
+        self.seq_offset = seq_offset  # a rank's sequences draw distinct sub-streams
+        dev = device
+
+        self.cache = kvq.KVCache(self.fmt, self.num_blocks, H, D, device=dev)
+        self.d_bt = torch.from_numpy(self.bt).to(dev)
+        self.d_lens = torch.from_numpy(self.lens).to(dev)
+        self.err = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.amax = torch.zeros(2, dtype=torch.float32, device=dev)
+        self.scales = torch.ones(2, dtype=torch.float32, device=dev)
+        self.d_ks, self.d_vs = self.scales[0:1], self.scales[1:2]
+
+        # calibration: the first calib_tokens tokens of sequence 0, or all tokens
+        if self.fmt != "bf16":
+            for b in range(B if w.calib_tokens is None else 1):
+                k, v = self.tokens(b)
+                n = L if w.calib_tokens is None else w.calib_tokens
+                kvq.kv_calibrate_absmax(k[:n].contiguous(), self.amax[0:1])
+                kvq.kv_calibrate_absmax(v[:n].contiguous(), self.amax[1:2])
+                del k, v
+            kvq.kv_scale_from_absmax_device(self.fmt, self.amax[0:1], self.d_ks)
+            kvq.kv_scale_from_absmax_device(self.fmt, self.amax[1:2], self.d_vs)
+
+        # fill the context (all but the step's chunk), keep the chunk for the step
+        step_k, step_v = [], []
+        ctx = L - self.chunk
+        for b in range(B):
+            k, v = self.tokens(b)
+            if ctx > 0:
+                slots = torch.from_numpy(wl.physical_slots(self.bt, b, np.arange(ctx))).to(dev)
+                kvq.kv_quantize_write(self.fmt, k[:ctx], v[:ctx], slots, self.cache, self.d_ks,
+                                      self.d_vs, self.err)
+            step_k.append(k[ctx:].clone())
+            step_v.append(v[ctx:].clone())
+            del k, v
+        self.step_k = torch.cat(step_k).contiguous()
+        self.step_v = torch.cat(step_v).contiguous()
+        # logical slots (seq * max_blocks * 16 + position) of the step's tokens,
+        # translated through the block table inside the write kernel
+        logical = np.concatenate([b * self.mb * wl.PAGE + np.arange(ctx, L) for b in range(B)])
+        self.step_slots = torch.from_numpy(logical.astype(np.int64)).to(dev)
+
+        g = torch.Generator(device=dev)
+        g.manual_seed(w.seed * 7919 + 17 + seq_offset)
+        self.q = torch.randn((B, Hq, D), generator=g, device=dev).to(torch.bfloat16)
+        self.out = torch.empty((B, Hq, D), dtype=torch.float32, device=dev)
+        self.lse = torch.empty((B, Hq), dtype=torch.float32, device=dev)
+        self.ws = kvq.new_workspace(
+            kvq.kv_decode_workspace_size(self.fmt, B, Hq, H, D, L), device=dev)
+        torch.cuda.synchronize()
+
+    def tokens(self, b: int):
+        """BF16 K and V ([L][H][D]) of sequence b (deterministic per workload)."""
+        s = 2 * (b + self.seq_offset)
+        k = wl.device_tokens(self.w.seed, s, self.L, self.H, self.D, self.out_k,
+                             self.w.outlier_factor, self.device)
+        v = wl.device_tokens(self.w.seed, s + 1, self.L, self.H, self.D, self.out_v,
+                             self.w.outlier_factor, self.device)
+        return k, v
+
+    @property
+    def scan_bytes(self) -> int:
+        return kv_scan_bytes(self.fmt, self.lens, self.H, self.D)
+
+    def write(self, stream=None):
+        kvq.kv_quantize_write(self.fmt, self.step_k, self.step_v, self.step_slots, self.cache,
+                              self.d_ks, self.d_vs, self.err, block_table=self.d_bt,
+                              stream=stream)
+
+    def decode(self, stream=None, q=None, out=None, lse=None):
+        kvq.kv_decode_attention(self.fmt, self.q if q is None else q, self.cache, self.d_bt,
+                                self.d_lens, self.L, self.d_ks, self.d_vs,
+                                self.out if out is None else out,
+                                self.lse if lse is None else lse, self.ws, self.err,
+                                stream=stream)
+
+    def step(self, stream=None):
+        self.write(stream)
+        self.decode(stream)

@@ -125,3 +125,29 @@ WORKLOADS = {
     "agents-fp8-4x127k": Workload("agents-fp8-4x127k", "fp8", 4, 8, 64, 128, 126976, 20263,
                                   {"frac": 0.01}, {"frac": 0.01}, 16.0, 16384, True, 2048),
 }
+
+
+def device_tokens(seed: int, stream: int, T: int, H: int, D: int,
+                  outliers: list[tuple[int, int]] = (), factor: float = 1.0,
+                  device: str = "cuda"):
+    """[T][H][D] bf16 on the device: N(0, 1) from torch's seeded CUDA generator
+    (sub-stream ``stream``), listed channels scaled by ``factor``, rounded to
+    BF16 (nearest even).  Used for the large workloads, which are too big to
+    draw on the host quickly."""
+    import torch
+
+    g = torch.Generator(device=device)
+    g.manual_seed(seed * 1000003 + stream)
+    x = torch.randn((T, H, D), generator=g, device=device, dtype=torch.float32)
+    for h, c in outliers:
+        x[:, h, c] *= factor
+    return x.to(torch.bfloat16)
+
+
+def outliers_for(w: "Workload", H: int, D: int, which: str) -> list[tuple[int, int]]:
+    """The workload's outlier pairs for K ("k") or V ("v")."""
+    spec = w.k_outliers if which == "k" else w.v_outliers
+    if not spec:
+        return []
+    return outlier_pairs(rng_for(w.seed, 100 if which == "k" else 101), H, D,
+                         per_head=spec.get("per_head"), frac=spec.get("frac"))
