@@ -200,6 +200,34 @@ kvq_status kv_decode_attention(int32_t fmt, const void* q, const kvq_cache* cach
                                void* workspace, size_t workspace_bytes, int32_t* d_err,
                                kvq_stream stream);
 
+/* kv_decode_attention without a caller workspace, for callers that cannot
+ * allocate device memory when they run a decode step (their device memory
+ * belongs to a fixed pool they must not bypass, they may not pay a
+ * cudaMalloc's latency and implicit synchronisation there, or their host
+ * hands them no scratch).  The pages' method has no counterpart of this call;
+ * it only changes where the scratch lives.
+ *   - Arguments and results are those of kv_decode_attention, minus the
+ *     workspace.  The call allocates nothing (no cudaMalloc, cudaFree or
+ *     allocating library routine).
+ *   - The scratch is one 8 MiB device array inside the library, held by every
+ *     GPU that loads the library until the process exits.  A problem whose
+ *     kv_decode_workspace_size exceeds 8 MiB returns KVQ_ERR_WORKSPACE and
+ *     launches nothing.
+ *   - The first call on a device looks the array's device address up (once,
+ *     with that device current); make that first call before any stream
+ *     capture.
+ *   - Every call on a device shares the one array and clears the part it
+ *     uses before launching (an extra memset on the stream).  Calls that
+ *     overlap on the GPU (different streams, no ordering between them) race
+ *     on the array and give wrong results; order them on one stream. */
+kvq_status kv_decode_attention_static_ws(int32_t fmt, const void* q, const kvq_cache* cache,
+                                         const int32_t* block_table, int32_t max_blocks,
+                                         const int32_t* seq_lens, int32_t num_seqs,
+                                         int32_t num_q_heads, int32_t max_seq_len,
+                                         int32_t num_splits, const float* d_k_scale,
+                                         const float* d_v_scale, float sm_scale, float* out,
+                                         float* lse, int32_t* d_err, kvq_stream stream);
+
 /* Dequantise the cache at the listed PHYSICAL slots (int64 [n]) into fp32
  * k_out, v_out [n][num_kv_heads][head_dim] (for checking; not on the decode
  * path).  Slots outside the cache set KVQ_DERR_SLOT and their rows are left

@@ -31,7 +31,8 @@ DERR_TIMEOUT = 0x10
 
 EXPORTS = ("kvq_status_string", "kvq_last_error", "kv_cache_bytes", "kv_scale_from_absmax",
            "kv_scale_from_absmax_device", "kv_calibrate_absmax", "kv_quantize_write",
-           "kv_decode_workspace_size", "kv_decode_attention", "kv_dequantize")
+           "kv_decode_workspace_size", "kv_decode_attention", "kv_decode_attention_static_ws",
+           "kv_dequantize")
 
 
 class KvqError(RuntimeError):
@@ -70,6 +71,8 @@ def lib() -> ctypes.CDLL:
             "kv_decode_workspace_size": [i32, i32, i32, i32, i32, i32, i32, ctypes.POINTER(sz)],
             "kv_decode_attention": [i32, P, CP, P, i32, P, i32, i32, i32, i32, P, P, f32, P, P,
                                     P, sz, P, P],
+            "kv_decode_attention_static_ws": [i32, P, CP, P, i32, P, i32, i32, i32, i32, P, P,
+                                              f32, P, P, P, P],
             "kv_dequantize": [i32, CP, P, i64, P, P, P, P, P, P],
         }
         for name, args in sigs.items():
@@ -190,6 +193,26 @@ def kv_decode_attention(fmt, q: torch.Tensor, cache: KVCache, block_table: torch
                                      num_splits, _ptr(k_scale), _ptr(v_scale), float(sm_scale),
                                      _ptr(out), _ptr(lse), _ptr(workspace), ws_bytes, _ptr(d_err),
                                      _stream(stream)))
+
+
+def kv_decode_attention_static_ws(fmt, q: torch.Tensor, cache: KVCache,
+                                  block_table: torch.Tensor, seq_lens: torch.Tensor,
+                                  max_seq_len: int, k_scale, v_scale, out: torch.Tensor,
+                                  lse: torch.Tensor | None, d_err: torch.Tensor | None = None,
+                                  sm_scale: float = 0.0, num_splits: int = 0, stream=None):
+    """kv_decode_attention with the library's built-in scratch instead of a
+    caller workspace, for callers that cannot allocate device memory at the
+    call (see include/kvq.h).  Calls on one device share that scratch: keep
+    them ordered on one stream."""
+    assert q.dtype == torch.bfloat16 and q.is_contiguous()
+    assert block_table.dtype == torch.int32 and seq_lens.dtype == torch.int32
+    assert out.dtype == torch.float32
+    B, Hq, _ = q.shape
+    _check(lib().kv_decode_attention_static_ws(_fmt(fmt), _ptr(q), cache.c, _ptr(block_table),
+                                               block_table.shape[1], _ptr(seq_lens), B, Hq,
+                                               max_seq_len, num_splits, _ptr(k_scale),
+                                               _ptr(v_scale), float(sm_scale), _ptr(out),
+                                               _ptr(lse), _ptr(d_err), _stream(stream)))
 
 
 def kv_dequantize(fmt, cache: KVCache, slots: torch.Tensor, k_scale, v_scale,

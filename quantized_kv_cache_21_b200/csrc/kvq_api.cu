@@ -194,6 +194,8 @@ kvq_status make_maps(int fmt, const kvq_cache* c, void* buf, CUtensorMap* tile, 
 }  // namespace
 
 namespace kvq {
+void set_last_error(const char* msg) { snprintf(g_err, sizeof(g_err), "%s", msg); }
+
 int num_sms() {
   int dev = 0, n = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 148;

@@ -69,5 +69,7 @@ cudaError_t launch_absmax(const uint16_t* x, int64_t n, float* d_amax, cudaStrea
 cudaError_t launch_scale(int fmt, const float* d_amax, float* d_scale, cudaStream_t stream);
 
 int num_sms();
+// Sets the text kvq_last_error() returns on this thread.
+void set_last_error(const char* msg);
 
 }  // namespace kvq
