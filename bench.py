@@ -9,7 +9,8 @@ the workload "fp8-paged-4x32k": 4 sequences x 32,768 tokens, 8 KV heads, 64
 query heads, head_dim 128, FP8 E4M3 cache in 16-token pages at a random
 permutation of the pool, per-layer scales calibrated on a 16,384-token sample.
 value = KV-scan bytes per step / device time per step (GB/s).  L2 is flushed
-(a 512 MiB write) before every timed step.
+before every timed step (a 512 MiB write, then a 256 MiB read so no dirty
+lines are left for the timed kernel to write back).
 
 Extra keys report the other rows: the BF16 vs FP8 vs NVFP4 comparison on the
 1 x 65,536-token, D 64 workload, the 4 x 126,976-token agent step (2,048-token
@@ -158,9 +159,14 @@ class Timer:
     def __init__(self, torch, clocks):
         self.torch, self.clocks = torch, clocks
         self.flush_buf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+        self.clean_buf = torch.zeros(L2_FLUSH_BYTES // 2, dtype=torch.uint8, device="cuda")
 
     def flush(self):
+        """Evict L2 (write 512 MiB), then read 256 MiB so L2 holds clean lines:
+        the timed step neither hits in L2 nor pays for another kernel's
+        dirty-line write-back."""
         self.flush_buf.fill_(1)
+        self.clean_buf.max()
 
     def run(self, parts, K, W):
         """parts: list of callables launched in order each step.  Returns the
@@ -257,7 +263,7 @@ def workload_config(w, fmt=None):
     return {"workload": w.name, "format": fmt or w.fmt, "num_seqs": w.B, "seq_len": w.seq_len,
             "kv_heads": w.Hkv, "q_heads": w.Hq, "head_dim": w.D, "block_size": 16,
             "block_table": "random permutation" if w.permuted else "in order",
-            "l2": "flushed (512 MiB write) before every timed step"}
+            "l2": "flushed before every timed step (512 MiB write, then 256 MiB read)"}
 
 
 def roofline(bytes_per_launch, ms_list, peak, peak_kind, traffic):
