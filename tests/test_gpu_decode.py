@@ -160,3 +160,15 @@ def test_host_side_errors():
                                 out, None, None)
     with pytest.raises(kvq.KvqError):  # GQA ratio must divide
         kvq.kv_decode_workspace_size("fp8", 1, 7, 2, 64, 100, 0)
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+@pytest.mark.parametrize("D", [64, 128])
+def test_variable_lengths_like_the_sweep(fmt, D):
+    """Sweep-style batch: lengths uniform in [L/2, L], GQA 8, automatic split."""
+    rng = wl.rng_for(5000 + D, 2)
+    lens = wl.varlen(rng, 8, 2048).tolist()
+    c = Case(fmt, 8, 2, 16, D, lens, seed=5100 + D, factor=16.0)
+    out, lse = c.decode()
+    assert int(c.err.item()) == 0
+    assert_attention_close(out, lse, *c.reference())
