@@ -504,34 +504,55 @@ __device__ __forceinline__ void item_block(const DecodeParams& p, const UnitTabl
 
 // Merge the per-CTA partials of unit u (slots u + c for c in [c_first,
 // c_first + n)) into out / lse; threads t of nthreads share the float4
-// columns.  One pass with a running maximum, so the loads of several partials
-// are in flight together.
+// columns.  Partials are read kBatch at a time with all their loads in
+// flight together: first the maxima, then the weighted sums.
 template <int D, int WPART>
 __device__ __forceinline__ void final_merge(const DecodeParams& p, int u, int b, int h, int grp,
                                             int c_first, int n, float vs, int t, int nthreads) {
   const float kInf = __int_as_float(0x7f800000);
+  constexpr int kBatch = 8;  // partials whose loads are in flight together
   const float* up = p.ws_part + (static_cast<size_t>(u) + c_first) * WPART;
   for (int col = t; col < 2 * D; col += nthreads) {  // float4 columns of [8][D]
     const int hh = col / (D / 4), d4 = (col - hh * (D / 4)) * 4;
     const int qi = grp * 8 + hh;
     if (qi >= p.G) continue;
-    float M = -kInf, L = 0.f;
+    float M = -kInf;
+    for (int s0 = 0; s0 < n; s0 += kBatch) {
+      float m[kBatch];
+#pragma unroll
+      for (int i = 0; i < kBatch; ++i)
+        m[i] = s0 + i < n ? __ldcg(up + (s0 + i) * WPART + hh) : -kInf;
+#pragma unroll
+      for (int i = 0; i < kBatch; ++i) M = fmaxf(M, m[i]);
+    }
+    float L = 0.f;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 4
-    for (int s = 0; s < n; ++s) {
-      const float* ps = up + s * WPART;
-      const float m = __ldcg(ps + hh);
-      const float l = __ldcg(ps + 8 + hh);
-      const float4 v4 = __ldcg(reinterpret_cast<const float4*>(ps + 16 + hh * D + d4));
-      if (m != -kInf) {
-        const float mn = fmaxf(M, m);
-        const float a = M == -kInf ? 0.f : fast_exp2(M - mn), e = fast_exp2(m - mn);
-        L = L * a + l * e;
-        acc.x = acc.x * a + v4.x * e;
-        acc.y = acc.y * a + v4.y * e;
-        acc.z = acc.z * a + v4.z * e;
-        acc.w = acc.w * a + v4.w * e;
-        M = mn;
+    if (M != -kInf) {
+      for (int s0 = 0; s0 < n; s0 += kBatch) {
+        float m[kBatch], l[kBatch];
+        float4 v4[kBatch];
+#pragma unroll
+        for (int i = 0; i < kBatch; ++i) {
+          if (s0 + i < n) {
+            const float* ps = up + (s0 + i) * WPART;
+            m[i] = __ldcg(ps + hh);
+            l[i] = __ldcg(ps + 8 + hh);
+            v4[i] = __ldcg(reinterpret_cast<const float4*>(ps + 16 + hh * D + d4));
+          } else {
+            m[i] = -kInf;
+            l[i] = 0.f;
+            v4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+          }
+        }
+#pragma unroll
+        for (int i = 0; i < kBatch; ++i) {
+          const float e = fast_exp2(m[i] - M);  // 0 for an empty partial (m = -inf)
+          L += e * l[i];
+          acc.x += e * v4[i].x;
+          acc.y += e * v4[i].y;
+          acc.z += e * v4[i].z;
+          acc.w += e * v4[i].w;
+        }
       }
     }
     const float sc = L > 0.f ? vs / (L * kPScale) : 0.f;
@@ -643,11 +664,10 @@ __global__ void __launch_bounds__(Shape<FMT, D>::NW * 32, 1)
     if (lane == 0) {
       tab.n = nu;
       tab.total = run;
-#pragma unroll 1
-      for (int i = 0; i < NW * NSW; ++i) mbar_init(&bars_all[i], 1);
-      mbar_init_fence();
     }
   }
+  if (lane < NSW) mbar_init(&bars[lane], 1);  // each warp its own stages
+  mbar_init_fence();
   __syncthreads();
   const int total = tab.total;
   const int n_local = warp < total ? (total - warp + NW - 1) / NW : 0;
