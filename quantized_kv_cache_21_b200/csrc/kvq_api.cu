@@ -177,18 +177,15 @@ kvq_status make_maps(int fmt, const kvq_cache* c, void* buf, CUtensorMap* tile, 
     *sf = *tile;
     return s;
   }
-  // NVFP4: head page = 16 rows of D/2 code bytes, then 16 * D/16 scale bytes
-  const cuuint64_t dims[4] = {D / 2, 16, H, nb};
+  // NVFP4: a head page is 16 rows of D/2 code bytes followed by 16 * D/16
+  // scale bytes, i.e. 18 rows of D/2 bytes: one box covers codes and scales.
+  const cuuint64_t dims[4] = {D / 2, 18, H, nb};
   const cuuint64_t str[3] = {D / 2, 9 * D, 9 * D * H};
-  const cuuint32_t box[4] = {(cuuint32_t)(D / 2), 16, 1, 1};
+  const cuuint32_t box[4] = {(cuuint32_t)(D / 2), 18, 1, 1};
   kvq_status s = encode(tile, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, buf, dims, str, box,
                         D == 64 ? CU_TENSOR_MAP_SWIZZLE_32B : CU_TENSOR_MAP_SWIZZLE_64B);
-  if (s != KVQ_OK) return s;
-  const cuuint64_t dims_s[3] = {D, H, nb};
-  const cuuint64_t str_s[2] = {9 * D, 9 * D * H};
-  const cuuint32_t box_s[3] = {(cuuint32_t)D, 1, 1};
-  return encode(sf, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, static_cast<uint8_t*>(buf) + 8 * D, dims_s,
-                str_s, box_s, CU_TENSOR_MAP_SWIZZLE_NONE);
+  *sf = *tile;
+  return s;
 }
 
 }  // namespace

@@ -273,21 +273,21 @@ __device__ __forceinline__ uint32_t scale_pair(uint32_t sa, uint32_t sb) {
   return lo;
 }
 
-// ---- NVFP4, head_dim 64: code rows of 32 B (32-byte swizzle) + 4 scale bytes.
+// ---- NVFP4, head_dim 64: a head page is 18 rows of 32 B, 16 code rows
+// (32-byte swizzle) then 2 rows of block scales (4 per token), fetched as one
+// box; the swizzle leaves rows 16-17 in place, so scales sit at byte 512.
 template <>
 struct Fmt<2, 64> {
   static constexpr bool kBF16 = false;
-  static constexpr int STAGE = 1280, TX = 1152, V_OFF = 512, KSF = 1024, VSF = 1152;
+  static constexpr int STAGE = 1536, TX = 1152, V_OFF = 768, KSF = 512, VSF = V_OFF + 512;
   __device__ static int k_elem(int tig, int i) { return 16 * tig + i; }
   __device__ static int v_elem(int gid, int i) { return 8 * gid + i; }
   __device__ static void issue(uint8_t* st, uint64_t* bar, const CUtensorMap* mk,
-                               const CUtensorMap* mv, const CUtensorMap* mks,
-                               const CUtensorMap* mvs, int h, int blk) {
+                               const CUtensorMap* mv, const CUtensorMap*, const CUtensorMap*,
+                               int h, int blk) {
     mbar_arrive_expect_tx(bar, TX);
     tma_load_4d(st, mk, bar, 0, 0, h, blk);
     tma_load_4d(st + V_OFF, mv, bar, 0, 0, h, blk);
-    tma_load_3d(st + KSF, mks, bar, 0, h, blk);
-    tma_load_3d(st + VSF, mvs, bar, 0, h, blk);
   }
   __device__ static void load_k(const uint8_t* st, int gid, int tig, uint32_t ka[4][4]) {
 #pragma unroll
@@ -335,21 +335,21 @@ struct Fmt<2, 64> {
   }
 };
 
-// ---- NVFP4, head_dim 128: code rows of 64 B (64-byte swizzle) + 8 scale bytes.
+// ---- NVFP4, head_dim 128: 18 rows of 64 B per head page, 16 code rows
+// (64-byte swizzle) then 2 scale rows (8 per token), one box; the scales stay
+// in place at byte 1024.  V starts at the next 512-byte swizzle repeat.
 template <>
 struct Fmt<2, 128> {
   static constexpr bool kBF16 = false;
-  static constexpr int STAGE = 2560, TX = 2304, V_OFF = 1024, KSF = 2048, VSF = 2176;
+  static constexpr int STAGE = 3072, TX = 2304, V_OFF = 1536, KSF = 1024, VSF = V_OFF + 1024;
   __device__ static int k_elem(int tig, int i) { return 32 * tig + i; }
   __device__ static int v_elem(int gid, int i) { return 16 * gid + i; }
   __device__ static void issue(uint8_t* st, uint64_t* bar, const CUtensorMap* mk,
-                               const CUtensorMap* mv, const CUtensorMap* mks,
-                               const CUtensorMap* mvs, int h, int blk) {
+                               const CUtensorMap* mv, const CUtensorMap*, const CUtensorMap*,
+                               int h, int blk) {
     mbar_arrive_expect_tx(bar, TX);
     tma_load_4d(st, mk, bar, 0, 0, h, blk);
     tma_load_4d(st + V_OFF, mv, bar, 0, 0, h, blk);
-    tma_load_3d(st + KSF, mks, bar, 0, h, blk);
-    tma_load_3d(st + VSF, mvs, bar, 0, h, blk);
   }
   __device__ static void load_k(const uint8_t* st, int gid, int tig, uint32_t ka[8][4]) {
 #pragma unroll
@@ -414,7 +414,7 @@ template <int FMT, int D>
 struct Shape {
   static constexpr int NW = (FMT == 0 && D == 128) ? 10 : 12;
   static constexpr int STAGE = Fmt<FMT, D>::STAGE;
-  static constexpr int NSW = STAGE <= 1280 ? 10 : STAGE <= 2048 ? 6 : STAGE <= 2560 ? 5
+  static constexpr int NSW = STAGE <= 1536 ? 10 : STAGE <= 2048 ? 6 : STAGE <= 3072 ? 4
                              : STAGE <= 4096 ? 3 : 2;
   static constexpr int WPART = 16 + 8 * D;  // floats of one partial: m[8], l[8], o[8][D]
 };
@@ -504,8 +504,8 @@ __device__ __forceinline__ void item_block(const DecodeParams& p, const UnitTabl
 
 // Merge the per-CTA partials of unit u (slots u + c for c in [c_first,
 // c_first + n)) into out / lse; threads t of nthreads share the float4
-// columns.  Partials are read kBatch at a time with all their loads in
-// flight together: first the maxima, then the weighted sums.
+// columns.  Partials are read kBatch at a time, all loads of a batch in
+// flight together (one pass when n <= kBatch), folded with a running max.
 template <int D, int WPART>
 __device__ __forceinline__ void final_merge(const DecodeParams& p, int u, int b, int h, int grp,
                                             int c_first, int n, float vs, int t, int nthreads) {
@@ -516,44 +516,44 @@ __device__ __forceinline__ void final_merge(const DecodeParams& p, int u, int b,
     const int hh = col / (D / 4), d4 = (col - hh * (D / 4)) * 4;
     const int qi = grp * 8 + hh;
     if (qi >= p.G) continue;
-    float M = -kInf;
-    for (int s0 = 0; s0 < n; s0 += kBatch) {
-      float m[kBatch];
-#pragma unroll
-      for (int i = 0; i < kBatch; ++i)
-        m[i] = s0 + i < n ? __ldcg(up + (s0 + i) * WPART + hh) : -kInf;
-#pragma unroll
-      for (int i = 0; i < kBatch; ++i) M = fmaxf(M, m[i]);
-    }
-    float L = 0.f;
+    float M = -kInf, L = 0.f;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (M != -kInf) {
-      for (int s0 = 0; s0 < n; s0 += kBatch) {
-        float m[kBatch], l[kBatch];
-        float4 v4[kBatch];
+    for (int s0 = 0; s0 < n; s0 += kBatch) {
+      float m[kBatch], l[kBatch];
+      float4 v4[kBatch];
 #pragma unroll
-        for (int i = 0; i < kBatch; ++i) {
-          if (s0 + i < n) {
-            const float* ps = up + (s0 + i) * WPART;
-            m[i] = __ldcg(ps + hh);
-            l[i] = __ldcg(ps + 8 + hh);
-            v4[i] = __ldcg(reinterpret_cast<const float4*>(ps + 16 + hh * D + d4));
-          } else {
-            m[i] = -kInf;
-            l[i] = 0.f;
-            v4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-          }
-        }
-#pragma unroll
-        for (int i = 0; i < kBatch; ++i) {
-          const float e = fast_exp2(m[i] - M);  // 0 for an empty partial (m = -inf)
-          L += e * l[i];
-          acc.x += e * v4[i].x;
-          acc.y += e * v4[i].y;
-          acc.z += e * v4[i].z;
-          acc.w += e * v4[i].w;
+      for (int i = 0; i < kBatch; ++i) {
+        if (s0 + i < n) {
+          const float* ps = up + (s0 + i) * WPART;
+          m[i] = __ldcg(ps + hh);
+          l[i] = __ldcg(ps + 8 + hh);
+          v4[i] = __ldcg(reinterpret_cast<const float4*>(ps + 16 + hh * D + d4));
+        } else {
+          m[i] = -kInf;
+          l[i] = 0.f;
+          v4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
         }
       }
+      float Mn = M;
+#pragma unroll
+      for (int i = 0; i < kBatch; ++i) Mn = fmaxf(Mn, m[i]);
+      if (Mn == -kInf) continue;  // nothing cached so far
+      const float a = fast_exp2(M - Mn);  // 0 while M = -inf
+      L *= a;
+      acc.x *= a;
+      acc.y *= a;
+      acc.z *= a;
+      acc.w *= a;
+#pragma unroll
+      for (int i = 0; i < kBatch; ++i) {
+        const float e = fast_exp2(m[i] - Mn);  // 0 for an empty partial (m = -inf)
+        L += e * l[i];
+        acc.x += e * v4[i].x;
+        acc.y += e * v4[i].y;
+        acc.z += e * v4[i].z;
+        acc.w += e * v4[i].w;
+      }
+      M = Mn;
     }
     const float sc = L > 0.f ? vs / (L * kPScale) : 0.f;
     const size_t row = static_cast<size_t>(b) * p.Hq + h * p.G + qi;
@@ -638,6 +638,21 @@ __global__ void __launch_bounds__(Shape<FMT, D>::NW * 32, 1)
   };
   load_q(u0);  // in flight while the unit table is built
 
+  // Block ids of this warp's first 64 local items, loaded now on the guess
+  // that they lie in unit u0 (they do unless its segment is shorter), so they
+  // share one memory round trip with q, the scales and seq_lens instead of
+  // waiting for the unit table.  Clamped to pmax - 1 <= max_blocks - 1, the
+  // loads stay in the table row; a wrong guess is discarded below.
+  const int g0 = warp + lane * NW, g1 = warp + (32 + lane) * NW;
+  int spec0, spec1;
+  {
+    const int32_t* bt0 = p.block_table +
+                         static_cast<size_t>(u0 / (p.n_groups * p.Hkv)) * p.max_blocks;
+    const int ps0 = ps_of(p, u0, vbeg);
+    spec0 = __ldg(bt0 + min(ps0 + g0, p.pmax - 1));
+    spec1 = __ldg(bt0 + min(ps0 + g1, p.pmax - 1));
+  }
+
   // ---- unit table: lane i of warp 0 looks at unit u0 + i (32 at a time)
   if (warp == 0) {
     int run = 0;
@@ -676,8 +691,21 @@ __global__ void __launch_bounds__(Shape<FMT, D>::NW * 32, 1)
   // items chunk + L (cur) and chunk + 32 + L (nxt).
   int chunk = 0;
   int cur_blk, cur_h, nxt_blk, nxt_h;
-  item_block(p, tab, u0, vbeg, vend, warp + lane * NW, cur_blk, cur_h);
-  item_block(p, tab, u0, vbeg, vend, warp + (32 + lane) * NW, nxt_blk, nxt_h);
+  {
+    const int k_first = tab.kend[0], h0 = (u0 / p.n_groups) % p.Hkv;
+    if (g0 < k_first) {
+      cur_blk = spec0;
+      cur_h = h0;
+    } else {
+      item_block(p, tab, u0, vbeg, vend, g0, cur_blk, cur_h);
+    }
+    if (g1 < k_first) {
+      nxt_blk = spec1;
+      nxt_h = h0;
+    } else {
+      item_block(p, tab, u0, vbeg, vend, g1, nxt_blk, nxt_h);
+    }
+  }
 
   // Issue the copies of local item i into stage i % NSW (all lanes call;
   // lane 0 issues).  stage_ok (warp-uniform) records which stages hold a
@@ -704,7 +732,22 @@ __global__ void __launch_bounds__(Shape<FMT, D>::NW * 32, 1)
       }
     }
   };
-  for (int i = 0; i < NSW && i < n_local; ++i) issue(i);
+  // Prologue: lane i fills stage i with local item i (its own cur_blk), the
+  // lanes' copies issued together rather than one after another.
+  {
+    const bool ok = cur_blk >= 0 && cur_blk < p.num_blocks;
+    const int n0 = min(NSW, n_local);
+    stage_ok = __ballot_sync(0xffffffffu, ok) & ((1u << n0) - 1u);
+    if (lane < n0) {
+      uint64_t* bar = &bars[lane];
+      if (ok) {
+        F::issue(ring + lane * F::STAGE, bar, &mk, &mv, &mks, &mvs, cur_h, cur_blk);
+      } else {
+        set_err(p.d_err, kErrBlockId);
+        mbar_arrive(bar);  // completes the phase with no data; the page is skipped
+      }
+    }
+  }
 
   const float c_log2 = p.sm_scale * ks * kLog2e;
   int k_base = 0, j = 0;  // j = this warp's next local item
@@ -902,16 +945,17 @@ __global__ void __launch_bounds__(Shape<FMT, D>::NW * 32, 1)
       }
     }
     if (!alone) {
-      // ---- the last CTA of the unit to get here merges all its partials
-      __threadfence();
+      // ---- the last CTA of the unit to get here merges all its partials.
+      // The barrier orders the CTA's partial stores before thread 0's
+      // release; its acquire, then the barrier, orders the merge's loads
+      // after every other CTA's release.
       __syncthreads();
       if (tid == 0) {
-        const unsigned t = atomicAdd(p.ws_cnt + u, 1u);
+        const unsigned t = atom_add_acq_rel_gpu(p.ws_cnt + u, 1u);
         s_last = (t == static_cast<unsigned>(c_last - c_first));
       }
       __syncthreads();
       if (s_last) {
-        __threadfence();
         final_merge<D, S::WPART>(p, u, b, h, grp, c_first, c_last - c_first + 1, vs, tid, NT);
         if (tid == 0) p.ws_cnt[u] = 0u;  // ready for the next launch
       }

@@ -18,6 +18,13 @@ constexpr int kErrScale = 0x4;
 constexpr int kErrSeqLen = 0x8;
 constexpr int kErrTimeout = 0x10;
 
+// Atomic add at GPU scope with acquire-release semantics; returns the old value.
+__device__ __forceinline__ unsigned atom_add_acq_rel_gpu(unsigned* p, unsigned v) {
+  unsigned old;
+  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+
 __device__ __forceinline__ void set_err(int* d_err, int bit) {
   if (d_err) atomicOr(d_err, bit);
 }
