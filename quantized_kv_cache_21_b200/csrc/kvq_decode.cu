@@ -85,23 +85,36 @@ struct Fmt<1, 128> {
     tma_load_4d(st, mk, bar, 0, 0, h, blk);
     tma_load_4d(st + V_OFF, mv, bar, 0, 0, h, blk);
   }
-  __device__ static void load_k(const uint8_t* st, int gid, int tig, uint32_t ka[8][4]) {
+  // Raw stage words of this thread: K rows gid, gid+8 (32 codes each), V
+  // rows 2tig, 2tig+1, 2tig+8, 2tig+9 (16 codes each).
+  struct Raw {
+    uint4 k[4], v[4];
+  };
+  static constexpr bool kLateV = false;
+  __device__ static void load_raw(const uint8_t* st, int gid, int tig, Raw& r) {
 #pragma unroll
-    for (int r = 0; r < 2; ++r) {
-      const int row = gid + 8 * r;
-      const uint4 a = lds128(st + swz128(row, 32 * tig));
-      const uint4 c = lds128(st + swz128(row, 32 * tig + 16));
+    for (int rr = 0; rr < 2; ++rr) {
+      const int row = gid + 8 * rr;
+      r.k[2 * rr] = lds128(st + swz128(row, 32 * tig));
+      r.k[2 * rr + 1] = lds128(st + swz128(row, 32 * tig + 16));
+    }
+    const uint8_t* sv = st + V_OFF;
+    r.v[0] = lds128(sv + swz128(2 * tig, 16 * gid));
+    r.v[1] = lds128(sv + swz128(2 * tig + 1, 16 * gid));
+    r.v[2] = lds128(sv + swz128(2 * tig + 8, 16 * gid));
+    r.v[3] = lds128(sv + swz128(2 * tig + 9, 16 * gid));
+  }
+  __device__ static void conv_k(const Raw& r, uint32_t ka[8][4]) {
+#pragma unroll
+    for (int rr = 0; rr < 2; ++rr) {
+      const uint4 a = r.k[2 * rr], c = r.k[2 * rr + 1];
       const uint32_t w[8] = {a.x, a.y, a.z, a.w, c.x, c.y, c.z, c.w};
 #pragma unroll
-      for (int s = 0; s < 8; ++s) e4m3x4_to_f16x2x2(w[s], ka[s][r], ka[s][2 + r]);
+      for (int s = 0; s < 8; ++s) e4m3x4_to_f16x2x2(w[s], ka[s][rr], ka[s][2 + rr]);
     }
   }
-  __device__ static void load_v(const uint8_t* st, int gid, int tig, uint32_t va[8][4]) {
-    const uint8_t* sv = st + V_OFF;
-    const uint4 X = lds128(sv + swz128(2 * tig, 16 * gid));
-    const uint4 Y = lds128(sv + swz128(2 * tig + 1, 16 * gid));
-    const uint4 Z = lds128(sv + swz128(2 * tig + 8, 16 * gid));
-    const uint4 W = lds128(sv + swz128(2 * tig + 9, 16 * gid));
+  __device__ static void conv_v(const Raw& r, uint32_t va[8][4]) {
+    const uint4 X = r.v[0], Y = r.v[1], Z = r.v[2], W = r.v[3];
     const uint32_t x[4] = {X.x, X.y, X.z, X.w}, y[4] = {Y.x, Y.y, Y.z, Y.w};
     const uint32_t z[4] = {Z.x, Z.y, Z.z, Z.w}, w[4] = {W.x, W.y, W.z, W.w};
 #pragma unroll
@@ -128,21 +141,31 @@ struct Fmt<1, 64> {
     tma_load_4d(st, mk, bar, 0, 0, h, blk);
     tma_load_4d(st + V_OFF, mv, bar, 0, 0, h, blk);
   }
-  __device__ static void load_k(const uint8_t* st, int gid, int tig, uint32_t ka[4][4]) {
+  struct Raw {
+    uint4 k[2];
+    uint2 v[4];
+  };
+  static constexpr bool kLateV = false;
+  __device__ static void load_raw(const uint8_t* st, int gid, int tig, Raw& r) {
 #pragma unroll
-    for (int r = 0; r < 2; ++r) {
-      const uint4 a = lds128(st + swz64(gid + 8 * r, 16 * tig));
+    for (int rr = 0; rr < 2; ++rr) r.k[rr] = lds128(st + swz64(gid + 8 * rr, 16 * tig));
+    const uint8_t* sv = st + V_OFF;
+    r.v[0] = lds64(sv + swz64(2 * tig, 8 * gid));
+    r.v[1] = lds64(sv + swz64(2 * tig + 1, 8 * gid));
+    r.v[2] = lds64(sv + swz64(2 * tig + 8, 8 * gid));
+    r.v[3] = lds64(sv + swz64(2 * tig + 9, 8 * gid));
+  }
+  __device__ static void conv_k(const Raw& r, uint32_t ka[4][4]) {
+#pragma unroll
+    for (int rr = 0; rr < 2; ++rr) {
+      const uint4 a = r.k[rr];
       const uint32_t w[4] = {a.x, a.y, a.z, a.w};
 #pragma unroll
-      for (int s = 0; s < 4; ++s) e4m3x4_to_f16x2x2(w[s], ka[s][r], ka[s][2 + r]);
+      for (int s = 0; s < 4; ++s) e4m3x4_to_f16x2x2(w[s], ka[s][rr], ka[s][2 + rr]);
     }
   }
-  __device__ static void load_v(const uint8_t* st, int gid, int tig, uint32_t va[4][4]) {
-    const uint8_t* sv = st + V_OFF;
-    const uint2 X = lds64(sv + swz64(2 * tig, 8 * gid));
-    const uint2 Y = lds64(sv + swz64(2 * tig + 1, 8 * gid));
-    const uint2 Z = lds64(sv + swz64(2 * tig + 8, 8 * gid));
-    const uint2 W = lds64(sv + swz64(2 * tig + 9, 8 * gid));
+  __device__ static void conv_v(const Raw& r, uint32_t va[4][4]) {
+    const uint2 X = r.v[0], Y = r.v[1], Z = r.v[2], W = r.v[3];
     const uint32_t x[2] = {X.x, X.y}, y[2] = {Y.x, Y.y}, z[2] = {Z.x, Z.y}, w[2] = {W.x, W.y};
 #pragma unroll
     for (int wi = 0; wi < 2; ++wi) {
@@ -168,26 +191,37 @@ struct Fmt<0, 64> {
     tma_load_4d(st, mk, bar, 0, 0, h, blk);
     tma_load_4d(st + V_OFF, mv, bar, 0, 0, h, blk);
   }
-  __device__ static void load_k(const uint8_t* st, int gid, int tig, uint32_t ka[4][4]) {
+  struct Raw {
+    uint4 k[4], v[4];
+  };
+  static constexpr bool kLateV = false;
+  __device__ static void load_raw(const uint8_t* st, int gid, int tig, Raw& r) {
 #pragma unroll
-    for (int r = 0; r < 2; ++r) {
-      const int row = gid + 8 * r;
-      const uint4 a = lds128(st + swz128(row, 32 * tig));
-      const uint4 c = lds128(st + swz128(row, 32 * tig + 16));
+    for (int rr = 0; rr < 2; ++rr) {
+      const int row = gid + 8 * rr;
+      r.k[2 * rr] = lds128(st + swz128(row, 32 * tig));
+      r.k[2 * rr + 1] = lds128(st + swz128(row, 32 * tig + 16));
+    }
+    const uint8_t* sv = st + V_OFF;
+    r.v[0] = lds128(sv + swz128(2 * tig, 16 * gid));
+    r.v[1] = lds128(sv + swz128(2 * tig + 1, 16 * gid));
+    r.v[2] = lds128(sv + swz128(2 * tig + 8, 16 * gid));
+    r.v[3] = lds128(sv + swz128(2 * tig + 9, 16 * gid));
+  }
+  __device__ static void conv_k(const Raw& r, uint32_t ka[4][4]) {
+#pragma unroll
+    for (int rr = 0; rr < 2; ++rr) {
+      const uint4 a = r.k[2 * rr], c = r.k[2 * rr + 1];
       const uint32_t w[8] = {a.x, a.y, a.z, a.w, c.x, c.y, c.z, c.w};
 #pragma unroll
       for (int s = 0; s < 4; ++s) {
-        ka[s][r] = w[2 * s];
-        ka[s][2 + r] = w[2 * s + 1];
+        ka[s][rr] = w[2 * s];
+        ka[s][2 + rr] = w[2 * s + 1];
       }
     }
   }
-  __device__ static void load_v(const uint8_t* st, int gid, int tig, uint32_t va[4][4]) {
-    const uint8_t* sv = st + V_OFF;
-    const uint4 X = lds128(sv + swz128(2 * tig, 16 * gid));
-    const uint4 Y = lds128(sv + swz128(2 * tig + 1, 16 * gid));
-    const uint4 Z = lds128(sv + swz128(2 * tig + 8, 16 * gid));
-    const uint4 W = lds128(sv + swz128(2 * tig + 9, 16 * gid));
+  __device__ static void conv_v(const Raw& r, uint32_t va[4][4]) {
+    const uint4 X = r.v[0], Y = r.v[1], Z = r.v[2], W = r.v[3];
     const uint32_t x[4] = {X.x, X.y, X.z, X.w}, y[4] = {Y.x, Y.y, Y.z, Y.w};
     const uint32_t z[4] = {Z.x, Z.y, Z.z, Z.w}, w[4] = {W.x, W.y, W.z, W.w};
 #pragma unroll
@@ -220,31 +254,52 @@ struct Fmt<0, 128> {
     tma_load_4d(st + V_OFF, mv, bar, 0, 0, h, blk);
     tma_load_4d(st + V_OFF + 2048, mv, bar, 64, 0, h, blk);
   }
-  __device__ static void load_k(const uint8_t* st, int gid, int tig, uint32_t ka[8][4]) {
+  struct Raw {
+    uint4 k[8], v[8];
+  };
+  // 64 raw registers would not fit beside the accumulators: K is read and
+  // used first, V read after the QK product (kLateV), then the stage refilled.
+  static constexpr bool kLateV = true;
+  __device__ static void load_raw_k(const uint8_t* st, int gid, int tig, Raw& r) {
 #pragma unroll
     for (int hf = 0; hf < 2; ++hf) {
 #pragma unroll
-      for (int r = 0; r < 2; ++r) {
-        const int row = gid + 8 * r;
-        const uint4 a = lds128(st + 2048 * hf + swz128(row, 32 * tig));
-        const uint4 c = lds128(st + 2048 * hf + swz128(row, 32 * tig + 16));
+      for (int rr = 0; rr < 2; ++rr) {
+        const int row = gid + 8 * rr;
+        r.k[4 * hf + 2 * rr] = lds128(st + 2048 * hf + swz128(row, 32 * tig));
+        r.k[4 * hf + 2 * rr + 1] = lds128(st + 2048 * hf + swz128(row, 32 * tig + 16));
+      }
+    }
+  }
+  __device__ static void load_raw_v(const uint8_t* st, int gid, int tig, Raw& r) {
+#pragma unroll
+    for (int hf = 0; hf < 2; ++hf) {
+      const uint8_t* sv = st + V_OFF + 2048 * hf;
+      r.v[4 * hf] = lds128(sv + swz128(2 * tig, 16 * gid));
+      r.v[4 * hf + 1] = lds128(sv + swz128(2 * tig + 1, 16 * gid));
+      r.v[4 * hf + 2] = lds128(sv + swz128(2 * tig + 8, 16 * gid));
+      r.v[4 * hf + 3] = lds128(sv + swz128(2 * tig + 9, 16 * gid));
+    }
+  }
+  __device__ static void conv_k(const Raw& r, uint32_t ka[8][4]) {
+#pragma unroll
+    for (int hf = 0; hf < 2; ++hf) {
+#pragma unroll
+      for (int rr = 0; rr < 2; ++rr) {
+        const uint4 a = r.k[4 * hf + 2 * rr], c = r.k[4 * hf + 2 * rr + 1];
         const uint32_t w[8] = {a.x, a.y, a.z, a.w, c.x, c.y, c.z, c.w};
 #pragma unroll
         for (int s = 0; s < 4; ++s) {
-          ka[4 * hf + s][r] = w[2 * s];
-          ka[4 * hf + s][2 + r] = w[2 * s + 1];
+          ka[4 * hf + s][rr] = w[2 * s];
+          ka[4 * hf + s][2 + rr] = w[2 * s + 1];
         }
       }
     }
   }
-  __device__ static void load_v(const uint8_t* st, int gid, int tig, uint32_t va[8][4]) {
+  __device__ static void conv_v(const Raw& r, uint32_t va[8][4]) {
 #pragma unroll
     for (int hf = 0; hf < 2; ++hf) {
-      const uint8_t* sv = st + V_OFF + 2048 * hf;
-      const uint4 X = lds128(sv + swz128(2 * tig, 16 * gid));
-      const uint4 Y = lds128(sv + swz128(2 * tig + 1, 16 * gid));
-      const uint4 Z = lds128(sv + swz128(2 * tig + 8, 16 * gid));
-      const uint4 W = lds128(sv + swz128(2 * tig + 9, 16 * gid));
+      const uint4 X = r.v[4 * hf], Y = r.v[4 * hf + 1], Z = r.v[4 * hf + 2], W = r.v[4 * hf + 3];
       const uint32_t x[4] = {X.x, X.y, X.z, X.w}, y[4] = {Y.x, Y.y, Y.z, Y.w};
       const uint32_t z[4] = {Z.x, Z.y, Z.z, Z.w}, w[4] = {W.x, W.y, W.z, W.w};
 #pragma unroll
@@ -289,34 +344,52 @@ struct Fmt<2, 64> {
     tma_load_4d(st, mk, bar, 0, 0, h, blk);
     tma_load_4d(st + V_OFF, mv, bar, 0, 0, h, blk);
   }
-  __device__ static void load_k(const uint8_t* st, int gid, int tig, uint32_t ka[4][4]) {
+  // Raw stage words: K code rows gid, gid+8 (16 codes each) and their block
+  // scale (block tig); V code rows 2tig, 2tig+1, 2tig+8, 2tig+9 (8 codes
+  // each, block gid/2) and the four scales.
+  struct Raw {
+    uint2 k[2];
+    uint32_t v[4], ks[2], vs[4];
+  };
+  static constexpr bool kLateV = false;
+  __device__ static void load_raw(const uint8_t* st, int gid, int tig, Raw& r) {
 #pragma unroll
-    for (int r = 0; r < 2; ++r) {
-      const int row = gid + 8 * r;
-      const uint2 c = lds64(st + swz32(row, 8 * tig));
-      const uint32_t sc = scale_pair(st[KSF + row * 4 + tig], st[KSF + row * 4 + tig]);
-      uint32_t f[8];
-      e2m1x8_to_f16x2x4(c.x, f);
-      e2m1x8_to_f16x2x4(c.y, f + 4);
-#pragma unroll
-      for (int s = 0; s < 4; ++s) {
-        ka[s][r] = hmul2(f[2 * s], sc);
-        ka[s][2 + r] = hmul2(f[2 * s + 1], sc);
-      }
+    for (int rr = 0; rr < 2; ++rr) {
+      const int row = gid + 8 * rr;
+      r.k[rr] = lds64(st + swz32(row, 8 * tig));
+      r.ks[rr] = st[KSF + row * 4 + tig];
     }
-  }
-  __device__ static void load_v(const uint8_t* st, int gid, int tig, uint32_t va[4][4]) {
     const uint8_t* sv = st + V_OFF;
     const uint8_t* ss = st + VSF;
     const int t0 = 2 * tig, t2 = 2 * tig + 8, blk = gid >> 1;
-    const uint32_t X = lds32(sv + swz32(t0, 4 * gid));
-    const uint32_t Y = lds32(sv + swz32(t0 + 1, 4 * gid));
-    const uint32_t Z = lds32(sv + swz32(t2, 4 * gid));
-    const uint32_t W = lds32(sv + swz32(t2 + 1, 4 * gid));
-    const uint32_t sxy = scale_pair(ss[t0 * 4 + blk], ss[(t0 + 1) * 4 + blk]);
-    const uint32_t szw = scale_pair(ss[t2 * 4 + blk], ss[(t2 + 1) * 4 + blk]);
+    r.v[0] = lds32(sv + swz32(t0, 4 * gid));
+    r.v[1] = lds32(sv + swz32(t0 + 1, 4 * gid));
+    r.v[2] = lds32(sv + swz32(t2, 4 * gid));
+    r.v[3] = lds32(sv + swz32(t2 + 1, 4 * gid));
+    r.vs[0] = ss[t0 * 4 + blk];
+    r.vs[1] = ss[(t0 + 1) * 4 + blk];
+    r.vs[2] = ss[t2 * 4 + blk];
+    r.vs[3] = ss[(t2 + 1) * 4 + blk];
+  }
+  __device__ static void conv_k(const Raw& r, uint32_t ka[4][4]) {
+#pragma unroll
+    for (int rr = 0; rr < 2; ++rr) {
+      const uint32_t sc = scale_pair(r.ks[rr], r.ks[rr]);
+      uint32_t f[8];
+      e2m1x8_to_f16x2x4(r.k[rr].x, f);
+      e2m1x8_to_f16x2x4(r.k[rr].y, f + 4);
+#pragma unroll
+      for (int s = 0; s < 4; ++s) {
+        ka[s][rr] = hmul2(f[2 * s], sc);
+        ka[s][2 + rr] = hmul2(f[2 * s + 1], sc);
+      }
+    }
+  }
+  __device__ static void conv_v(const Raw& r, uint32_t va[4][4]) {
+    const uint32_t sxy = scale_pair(r.vs[0], r.vs[1]);
+    const uint32_t szw = scale_pair(r.vs[2], r.vs[3]);
     uint32_t lo, hi, L[4], H[4];
-    nib_interleave(X, Y, lo, hi);
+    nib_interleave(r.v[0], r.v[1], lo, hi);
     e2m1x8_to_f16x2x4(lo, L);
     e2m1x8_to_f16x2x4(hi, H);
 #pragma unroll
@@ -324,7 +397,7 @@ struct Fmt<2, 64> {
       va[j][0] = hmul2(L[j], sxy);
       va[j][1] = hmul2(H[j], sxy);
     }
-    nib_interleave(Z, W, lo, hi);
+    nib_interleave(r.v[2], r.v[3], lo, hi);
     e2m1x8_to_f16x2x4(lo, L);
     e2m1x8_to_f16x2x4(hi, H);
 #pragma unroll
@@ -351,13 +424,41 @@ struct Fmt<2, 128> {
     tma_load_4d(st, mk, bar, 0, 0, h, blk);
     tma_load_4d(st + V_OFF, mv, bar, 0, 0, h, blk);
   }
-  __device__ static void load_k(const uint8_t* st, int gid, int tig, uint32_t ka[8][4]) {
+  // Raw stage words: K code rows gid, gid+8 (32 codes each) with their two
+  // block scales (blocks 2tig, 2tig+1, one 16-bit load); V code rows 2tig,
+  // 2tig+1, 2tig+8, 2tig+9 (16 codes each, block gid) and the four scales.
+  struct Raw {
+    uint4 k[2];
+    uint2 v[4];
+    uint32_t ks[2], vs[4];
+  };
+  static constexpr bool kLateV = false;
+  __device__ static void load_raw(const uint8_t* st, int gid, int tig, Raw& r) {
 #pragma unroll
-    for (int r = 0; r < 2; ++r) {
-      const int row = gid + 8 * r;
-      const uint4 c = lds128(st + swz64(row, 16 * tig));
-      const uint32_t s01 = scale_pair(st[KSF + row * 8 + 2 * tig], st[KSF + row * 8 + 2 * tig + 1]);
+    for (int rr = 0; rr < 2; ++rr) {
+      const int row = gid + 8 * rr;
+      r.k[rr] = lds128(st + swz64(row, 16 * tig));
+      r.ks[rr] = *reinterpret_cast<const uint16_t*>(st + KSF + row * 8 + 2 * tig);
+    }
+    const uint8_t* sv = st + V_OFF;
+    const uint8_t* ss = st + VSF;
+    const int t0 = 2 * tig, t2 = 2 * tig + 8;
+    r.v[0] = lds64(sv + swz64(t0, 8 * gid));
+    r.v[1] = lds64(sv + swz64(t0 + 1, 8 * gid));
+    r.v[2] = lds64(sv + swz64(t2, 8 * gid));
+    r.v[3] = lds64(sv + swz64(t2 + 1, 8 * gid));
+    r.vs[0] = ss[t0 * 8 + gid];
+    r.vs[1] = ss[(t0 + 1) * 8 + gid];
+    r.vs[2] = ss[t2 * 8 + gid];
+    r.vs[3] = ss[(t2 + 1) * 8 + gid];
+  }
+  __device__ static void conv_k(const Raw& r, uint32_t ka[8][4]) {
+#pragma unroll
+    for (int rr = 0; rr < 2; ++rr) {
+      uint32_t s01, unused;
+      e4m3x4_to_f16x2x2(r.ks[rr], s01, unused);  // (scale of block 2tig, of 2tig+1)
       const uint32_t sc0 = prmt(s01, s01, 0x1010), sc1 = prmt(s01, s01, 0x3232);
+      const uint4 c = r.k[rr];
       uint32_t f[16];
       e2m1x8_to_f16x2x4(c.x, f);
       e2m1x8_to_f16x2x4(c.y, f + 4);
@@ -366,22 +467,16 @@ struct Fmt<2, 128> {
 #pragma unroll
       for (int s = 0; s < 8; ++s) {
         const uint32_t sc = s < 4 ? sc0 : sc1;
-        ka[s][r] = hmul2(f[2 * s], sc);
-        ka[s][2 + r] = hmul2(f[2 * s + 1], sc);
+        ka[s][rr] = hmul2(f[2 * s], sc);
+        ka[s][2 + rr] = hmul2(f[2 * s + 1], sc);
       }
     }
   }
-  __device__ static void load_v(const uint8_t* st, int gid, int tig, uint32_t va[8][4]) {
-    const uint8_t* sv = st + V_OFF;
-    const uint8_t* ss = st + VSF;
-    const int t0 = 2 * tig, t2 = 2 * tig + 8;
-    const uint2 X = lds64(sv + swz64(t0, 8 * gid));
-    const uint2 Y = lds64(sv + swz64(t0 + 1, 8 * gid));
-    const uint2 Z = lds64(sv + swz64(t2, 8 * gid));
-    const uint2 W = lds64(sv + swz64(t2 + 1, 8 * gid));
-    const uint32_t sxy = scale_pair(ss[t0 * 8 + gid], ss[(t0 + 1) * 8 + gid]);
-    const uint32_t szw = scale_pair(ss[t2 * 8 + gid], ss[(t2 + 1) * 8 + gid]);
-    const uint32_t x[2] = {X.x, X.y}, y[2] = {Y.x, Y.y}, z[2] = {Z.x, Z.y}, w[2] = {W.x, W.y};
+  __device__ static void conv_v(const Raw& r, uint32_t va[8][4]) {
+    const uint32_t sxy = scale_pair(r.vs[0], r.vs[1]);
+    const uint32_t szw = scale_pair(r.vs[2], r.vs[3]);
+    const uint32_t x[2] = {r.v[0].x, r.v[0].y}, y[2] = {r.v[1].x, r.v[1].y};
+    const uint32_t z[2] = {r.v[2].x, r.v[2].y}, w[2] = {r.v[3].x, r.v[3].y};
 #pragma unroll
     for (int wi = 0; wi < 2; ++wi) {
       uint32_t lo, hi, L[4], H[4];
@@ -405,17 +500,18 @@ struct Fmt<2, 128> {
   }
 };
 
-// Kernel shape per format: warps per CTA and stages per warp.
 // Kernel shape per format: warps per CTA (NW, one CTA per SM) and ring stages
-// per warp (NSW).  Each warp owns NSW stages (~150 KB of ring per SM in all)
-// and refills a stage only after consuming it, so every mbarrier wait is
+// per warp (NSW).  Each warp owns NSW stages (~150-170 KB of ring per SM in
+// all) and refills a stage only after consuming it, so every mbarrier wait is
 // exactly one phase ahead; NW warp-partial slots serve the segment merge.
+// The quantized head_dim-64 pages are small and their scan is bound by
+// instruction latency, so those kernels run 16 warps (128 registers each).
 template <int FMT, int D>
 struct Shape {
-  static constexpr int NW = (FMT == 0 && D == 128) ? 10 : 12;
+  static constexpr int NW = (FMT != 0 && D == 64) ? 16 : (FMT == 0 && D == 128) ? 10 : 12;
   static constexpr int STAGE = Fmt<FMT, D>::STAGE;
-  static constexpr int NSW = STAGE <= 1536 ? 10 : STAGE <= 2048 ? 6 : STAGE <= 3072 ? 4
-                             : STAGE <= 4096 ? 3 : 2;
+  static constexpr int NSW = (FMT == 2 && D == 64) ? 7 : (FMT == 1 && D == 64) ? 5
+                             : STAGE <= 2048 ? 6 : STAGE <= 3072 ? 4 : STAGE <= 4096 ? 3 : 2;
   static constexpr int WPART = 16 + 8 * D;  // floats of one partial: m[8], l[8], o[8][D]
 };
 
@@ -793,11 +889,15 @@ __global__ void __launch_bounds__(Shape<FMT, D>::NW * 32, 1)
       const int n_valid = min(kPage, len - page * kPage);
       const bool valid = (stage_ok >> st) & 1u;
 
+      // The stage's words go to registers first, so the stage is refilled with
+      // local item j + NSW before any decode or math on this one (for BF16
+      // head_dim 128, after the QK product: see kLateV).
+      typename F::Raw raw;
       uint32_t ka[KS][4], va[MT][4];
       float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
-      if (valid) {
-        // ---- S^T = K Q^T on tensor cores (two accumulator chains)
-        F::load_k(sp, gid, tig, ka);
+      // ---- S^T = K Q^T on tensor cores (two accumulator chains)
+      auto qk = [&]() {
+        F::conv_k(raw, ka);
 #pragma unroll
         for (int s = 0; s < KS; ++s) {
           if (s & 1)
@@ -805,15 +905,24 @@ __global__ void __launch_bounds__(Shape<FMT, D>::NW * 32, 1)
           else
             mma16816<F::kBF16>(sa, ka[s], qb[s][0], qb[s][1]);
         }
-        F::load_v(sp, gid, tig, va);
+      };
+      if constexpr (F::kLateV) {
+        if (valid) {
+          F::load_raw_k(sp, gid, tig, raw);
+          qk();
+          F::load_raw_v(sp, gid, tig, raw);
+        }
+      } else if (valid) {
+        F::load_raw(sp, gid, tig, raw);
       }
-      // the stage is in registers: refill it with local item j + NSW
       __syncwarp();
       if (j + NSW < n_local) {
         if (lane == 0) fence_proxy_async_smem();
         issue(j + NSW);
       }
       if (!valid) continue;
+      if constexpr (!F::kLateV) qk();
+      F::conv_v(raw, va);
 
       float s0 = (sa[0] + sb[0]) * c_log2, s1 = (sa[1] + sb[1]) * c_log2;
       float s2 = (sa[2] + sb[2]) * c_log2, s3 = (sa[3] + sb[3]) * c_log2;
