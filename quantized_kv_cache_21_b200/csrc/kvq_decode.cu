@@ -85,6 +85,10 @@ struct Fmt<1, 128> {
     tma_load_4d(st, mk, bar, 0, 0, h, blk);
     tma_load_4d(st + V_OFF, mv, bar, 0, 0, h, blk);
   }
+  __device__ static void prefetch(const CUtensorMap* mk, const CUtensorMap* mv, int h, int blk) {
+    tma_prefetch_l2_4d(mk, 0, 0, h, blk);
+    tma_prefetch_l2_4d(mv, 0, 0, h, blk);
+  }
   // Raw stage words of this thread: K rows gid, gid+8 (32 codes each), V
   // rows 2tig, 2tig+1, 2tig+8, 2tig+9 (16 codes each).
   struct Raw {
@@ -141,6 +145,10 @@ struct Fmt<1, 64> {
     tma_load_4d(st, mk, bar, 0, 0, h, blk);
     tma_load_4d(st + V_OFF, mv, bar, 0, 0, h, blk);
   }
+  __device__ static void prefetch(const CUtensorMap* mk, const CUtensorMap* mv, int h, int blk) {
+    tma_prefetch_l2_4d(mk, 0, 0, h, blk);
+    tma_prefetch_l2_4d(mv, 0, 0, h, blk);
+  }
   struct Raw {
     uint4 k[2];
     uint2 v[4];
@@ -190,6 +198,10 @@ struct Fmt<0, 64> {
     mbar_arrive_expect_tx(bar, TX);
     tma_load_4d(st, mk, bar, 0, 0, h, blk);
     tma_load_4d(st + V_OFF, mv, bar, 0, 0, h, blk);
+  }
+  __device__ static void prefetch(const CUtensorMap* mk, const CUtensorMap* mv, int h, int blk) {
+    tma_prefetch_l2_4d(mk, 0, 0, h, blk);
+    tma_prefetch_l2_4d(mv, 0, 0, h, blk);
   }
   struct Raw {
     uint4 k[4], v[4];
@@ -253,6 +265,12 @@ struct Fmt<0, 128> {
     tma_load_4d(st + 2048, mk, bar, 64, 0, h, blk);
     tma_load_4d(st + V_OFF, mv, bar, 0, 0, h, blk);
     tma_load_4d(st + V_OFF + 2048, mv, bar, 64, 0, h, blk);
+  }
+  __device__ static void prefetch(const CUtensorMap* mk, const CUtensorMap* mv, int h, int blk) {
+    tma_prefetch_l2_4d(mk, 0, 0, h, blk);
+    tma_prefetch_l2_4d(mk, 64, 0, h, blk);
+    tma_prefetch_l2_4d(mv, 0, 0, h, blk);
+    tma_prefetch_l2_4d(mv, 64, 0, h, blk);
   }
   struct Raw {
     uint4 k[8], v[8];
@@ -344,6 +362,10 @@ struct Fmt<2, 64> {
     tma_load_4d(st, mk, bar, 0, 0, h, blk);
     tma_load_4d(st + V_OFF, mv, bar, 0, 0, h, blk);
   }
+  __device__ static void prefetch(const CUtensorMap* mk, const CUtensorMap* mv, int h, int blk) {
+    tma_prefetch_l2_4d(mk, 0, 0, h, blk);
+    tma_prefetch_l2_4d(mv, 0, 0, h, blk);
+  }
   // Raw stage words: K code rows gid, gid+8 (16 codes each) and their block
   // scale (block tig); V code rows 2tig, 2tig+1, 2tig+8, 2tig+9 (8 codes
   // each, block gid/2) and the four scales.
@@ -423,6 +445,10 @@ struct Fmt<2, 128> {
     mbar_arrive_expect_tx(bar, TX);
     tma_load_4d(st, mk, bar, 0, 0, h, blk);
     tma_load_4d(st + V_OFF, mv, bar, 0, 0, h, blk);
+  }
+  __device__ static void prefetch(const CUtensorMap* mk, const CUtensorMap* mv, int h, int blk) {
+    tma_prefetch_l2_4d(mk, 0, 0, h, blk);
+    tma_prefetch_l2_4d(mv, 0, 0, h, blk);
   }
   // Raw stage words: K code rows gid, gid+8 (32 codes each) with their two
   // block scales (blocks 2tig, 2tig+1, one 16-bit load); V code rows 2tig,
@@ -682,6 +708,10 @@ __global__ void __launch_bounds__(Shape<FMT, D>::NW * 32, 1)
   const int gid = lane >> 2, tig = lane & 3;
   const int c = blockIdx.x, C = gridDim.x;
   const int64_t V = static_cast<int64_t>(p.units) * p.pmax;
+  if (tid == 0) {
+    tma_prefetch_desc(&mk);
+    tma_prefetch_desc(&mv);
+  }
   uint8_t* ring = rings + static_cast<size_t>(warp) * NSW * F::STAGE;
   uint64_t* bars = bars_all + warp * NSW;
 
@@ -777,9 +807,17 @@ __global__ void __launch_bounds__(Shape<FMT, D>::NW * 32, 1)
       tab.total = run;
     }
   }
+  // Ask L2 for the pages of this warp's first stages (the guessed block ids)
+  // while the unit table is built; a wrong guess only costs a prefetch.
+  if (lane < NSW && spec0 >= 0 && spec0 < p.num_blocks)
+    F::prefetch(&mk, &mv, (u0 / p.n_groups) % p.Hkv, spec0);
   if (lane < NSW) mbar_init(&bars[lane], 1);  // each warp its own stages
   mbar_init_fence();
   __syncthreads();
+  // Everything read so far (q, tables, scales) predates a preceding cache
+  // write of this stream; its cache stores must be visible before the first
+  // page copy (this launch may overlap that write's tail).
+  griddep_wait();
   const int total = tab.total;
   const int n_local = warp < total ? (total - warp + NW - 1) / NW : 0;
 
@@ -1093,9 +1131,19 @@ cudaError_t launch_t(const CUtensorMap* maps, const DecodeParams& p, int ctas,
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  kvq_decode_kernel<FMT, D><<<ctas, S::NW * 32, smem, stream>>>(maps[0], maps[1], maps[2],
-                                                               maps[3], p);
-  return cudaGetLastError();
+  // Programmatic stream serialization: the launch may begin while a
+  // preceding kv_quantize_write of this stream finishes (see griddep_wait).
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(ctas);
+  cfg.blockDim = dim3(S::NW * 32);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kvq_decode_kernel<FMT, D>, maps[0], maps[1], maps[2], maps[3], p);
 }
 
 template <int FMT, int D>

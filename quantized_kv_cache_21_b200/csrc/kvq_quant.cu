@@ -48,6 +48,7 @@ __device__ __forceinline__ int64_t resolve_slot(const QuantParams& p, int64_t t)
 
 // One thread = 8 elements of one (token, K|V, head) row.
 __global__ void quantize_fp8_kernel(const QuantParams p) {
+  griddep_launch_dependents();  // a following decode may start its prologue
   const int cpr = p.D / 8;  // chunks per row
   const int64_t total = p.T * 2 * p.H * cpr;
   const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
@@ -79,6 +80,7 @@ __global__ void quantize_fp8_kernel(const QuantParams p) {
 
 // One thread = one 16-element block of one (token, K|V, head) row.
 __global__ void quantize_nvfp4_kernel(const QuantParams p) {
+  griddep_launch_dependents();  // a following decode may start its prologue
   const int bpr = p.D / 16;  // blocks per row
   const int64_t total = p.T * 2 * p.H * bpr;
   const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
@@ -130,6 +132,7 @@ __global__ void quantize_nvfp4_kernel(const QuantParams p) {
 
 // One thread = 8 elements (16 bytes) of one (token, K|V, head) row.
 __global__ void write_bf16_kernel(const QuantParams p) {
+  griddep_launch_dependents();  // a following decode may start its prologue
   const int cpr = p.D / 8;
   const int64_t total = p.T * 2 * p.H * cpr;
   const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;

@@ -9,7 +9,7 @@ import torch
 import quantized_kv_cache_21_b200 as kvq
 from quantized_kv_cache_21_b200 import workloads as wl
 
-from gpu_common import DEV, Case, assert_attention_close, dev_scalar, new_err
+from gpu_common import DEV, Case, assert_attention_close, dev_scalar, new_err, to_dev_bits
 
 pytestmark = pytest.mark.gpu
 
@@ -148,15 +148,16 @@ def test_bad_block_id_and_seq_len_are_reported():
 
 
 def test_host_side_errors():
-    c = Case("fp8", 1, 1, 8, 64, [1000], seed=4800)
-    need = kvq.kv_decode_workspace_size("fp8", 1, 8, 1, 64, 1008, 0)
+    # long enough that the automatic split spreads the one unit over CTAs
+    c = Case("fp8", 1, 1, 8, 64, [4000], seed=4800)
+    need = kvq.kv_decode_workspace_size("fp8", 1, 8, 1, 64, 4000, 0)
     assert need > 0
     out = torch.empty(1, 8, 64, device=DEV)
     with pytest.raises(kvq.KvqError, match="workspace"):
-        kvq.kv_decode_attention("fp8", c.d_q, c.cache, c.d_bt, c.d_lens, 1008, c.d_ks, c.d_vs,
+        kvq.kv_decode_attention("fp8", c.d_q, c.cache, c.d_bt, c.d_lens, 4000, c.d_ks, c.d_vs,
                                 out, None, kvq.new_workspace(need - 256 if need > 512 else 0))
     with pytest.raises(kvq.KvqError, match="max_seq_len"):
-        kvq.kv_decode_attention("fp8", c.d_q, c.cache, c.d_bt, c.d_lens, 1009, c.d_ks, c.d_vs,
+        kvq.kv_decode_attention("fp8", c.d_q, c.cache, c.d_bt, c.d_lens, 4001, c.d_ks, c.d_vs,
                                 out, None, None)
     with pytest.raises(kvq.KvqError):  # GQA ratio must divide
         kvq.kv_decode_workspace_size("fp8", 1, 7, 2, 64, 100, 0)
@@ -172,3 +173,47 @@ def test_variable_lengths_like_the_sweep(fmt, D):
     out, lse = c.decode()
     assert int(c.err.item()) == 0
     assert_attention_close(out, lse, *c.reference())
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+@pytest.mark.parametrize("D", [64, 128])
+def test_decode_launched_right_after_a_write(fmt, D):
+    """The decode may begin while a kv_quantize_write just before it on the
+    stream is finishing: the last 1,200 tokens of every sequence are written
+    and the decode launched next, with no other work between, and the result
+    must include them."""
+    lens = [3000, 2600, 1500]
+    c = Case(fmt, 3, 2, 16, D, lens, seed=5300 + D, factor=16.0)
+    tail = 1200
+    # rewrite the tails with fresh codes from zeroed pages: clear them first
+    kb = [torch.from_numpy(wl.physical_slots(c.bt, b, np.arange(n - tail, n))).to(DEV)
+          for b, n in enumerate(lens)]
+    page = kvq.kv_cache_bytes(fmt, 1, c.Hkv, D)
+    for b, n in enumerate(lens):
+        for blk in set(int(x) for x in c.bt[b][(n - tail) // 16:]):
+            c.cache.k[blk * page:(blk + 1) * page].zero_()
+            c.cache.v[blk * page:(blk + 1) * page].zero_()
+    # the head of the last page before the tail is zeroed too: write it back
+    msl = c.max_blocks * 16
+    ws = kvq.new_workspace(kvq.kv_decode_workspace_size(fmt, c.B, c.Hq, c.Hkv, D, msl))
+    out = torch.empty((c.B, c.Hq, D), device=DEV)
+    lse = torch.empty((c.B, c.Hq), device=DEV)
+    heads = [torch.from_numpy(wl.physical_slots(c.bt, b, np.arange((n - tail) // 16 * 16,
+                                                                  n - tail))).to(DEV)
+             for b, n in enumerate(lens)]
+    k_tail = torch.cat([to_dev_bits(c.k[b][n - tail:]) for b, n in enumerate(lens)])
+    v_tail = torch.cat([to_dev_bits(c.v[b][n - tail:]) for b, n in enumerate(lens)])
+    k_head = torch.cat([to_dev_bits(c.k[b][(n - tail) // 16 * 16:n - tail])
+                        for b, n in enumerate(lens)])
+    v_head = torch.cat([to_dev_bits(c.v[b][(n - tail) // 16 * 16:n - tail])
+                        for b, n in enumerate(lens)])
+    kvq.kv_quantize_write(fmt, k_head, v_head, torch.cat(heads), c.cache, c.d_ks, c.d_vs, c.err)
+    slots = torch.cat(kb)
+    torch.cuda.synchronize()
+    # write, then decode: adjacent launches on one stream
+    kvq.kv_quantize_write(fmt, k_tail, v_tail, slots, c.cache, c.d_ks, c.d_vs, c.err)
+    kvq.kv_decode_attention(fmt, c.d_q, c.cache, c.d_bt, c.d_lens, msl, c.d_ks, c.d_vs, out, lse,
+                            ws, c.err)
+    torch.cuda.synchronize()
+    assert int(c.err.item()) == 0
+    assert_attention_close(out.cpu().numpy(), lse.cpu().numpy(), *c.reference())
