@@ -46,109 +46,190 @@ __device__ __forceinline__ int64_t resolve_slot(const QuantParams& p, int64_t t)
   return s;
 }
 
-// One thread = 8 elements of one (token, K|V, head) row.
-__global__ void quantize_fp8_kernel(const QuantParams p) {
-  griddep_launch_dependents();  // a following decode may start its prologue
-  const int cpr = p.D / 8;  // chunks per row
-  const int64_t total = p.T * 2 * p.H * cpr;
-  const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (idx >= total) return;
-  const int c = static_cast<int>(idx % cpr);
-  int64_t r = idx / cpr;
-  const int h = static_cast<int>(r % p.H);
-  r /= p.H;
-  const int kv = static_cast<int>(r & 1);
-  const int64_t t = r >> 1;
-  const float s = __ldg(kv ? p.v_scale : p.k_scale);
-  if (!(s > 0.f && s < kInf)) {
-    if (idx == 0 || idx == cpr * p.H) set_err(p.d_err, kErrScale);
-    return;
-  }
-  const int64_t slot = resolve_slot(p, t);
-  if (slot < 0) return;
-  const uint16_t* src = (kv ? p.v : p.k) + (t * p.H + h) * p.D + 8 * c;
-  const uint4 x = __ldg(reinterpret_cast<const uint4*>(src));
-  const uint32_t w[4] = {x.x, x.y, x.z, x.w};
-  uint32_t code[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-    code[i] = f32x2_to_e4m3x2(__fdiv_rn(bf16_lo(w[i]), s), __fdiv_rn(bf16_hi(w[i]), s));
-  uint8_t* dst = (kv ? p.vc : p.kc) +
-                 ((slot / kPage * p.H + h) * kPage + slot % kPage) * p.D + 8 * c;
-  *reinterpret_cast<uint2*>(dst) = make_uint2(code[0] | (code[1] << 16), code[2] | (code[3] << 16));
+// The write kernels give each block `tpb` (<= kTokPerBlock) tokens, grid-
+// strided: the block's first threads resolve the tokens' slots in parallel
+// (one dependent load chain per block), then every thread takes chunks of
+// the tokens' 2 (K, V) x H rows x (D/8 or D/16) columns, kBatch (NVFP4:
+// kBatchNv) at a time with all their loads issued before any convert or store.
+constexpr int kTokPerBlock = 8;
+constexpr int kBatch = 4;
+constexpr int kBatchNv = 2;  // NVFP4 chunks hold 2x the registers
+
+struct TokSlots {
+  int64_t slot[kTokPerBlock];
+};
+
+__device__ __forceinline__ void block_slots(const QuantParams& p, int64_t t0, int tpb,
+                                            TokSlots& s) {
+  if (threadIdx.x < tpb)
+    s.slot[threadIdx.x] = t0 + threadIdx.x < p.T ? resolve_slot(p, t0 + threadIdx.x) : -1;
+  __syncthreads();
 }
 
-// One thread = one 16-element block of one (token, K|V, head) row.
-__global__ void quantize_nvfp4_kernel(const QuantParams p) {
+// Chunk ii of the block's tokens: token tt, K or V (kv), head h, column c.
+struct Chunk {
+  int64_t t, slot;
+  int kv, h, c;
+};
+__device__ __forceinline__ Chunk chunk_of(const TokSlots& ts, int64_t t0, int ii, int n,
+                                          int per_kv, int lg) {
+  Chunk q;
+  const int tt = ii / n, i = ii - tt * n;
+  q.t = t0 + tt;
+  q.slot = ts.slot[tt];
+  q.kv = i >= per_kv;
+  const int j = i - q.kv * per_kv;
+  q.h = j >> lg;
+  q.c = j & ((1 << lg) - 1);
+  return q;
+}
+
+// One chunk = 8 elements of one (K|V, head) row of a token.
+__global__ void quantize_fp8_kernel(const QuantParams p, int tpb) {
   griddep_launch_dependents();  // a following decode may start its prologue
-  const int bpr = p.D / 16;  // blocks per row
-  const int64_t total = p.T * 2 * p.H * bpr;
-  const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (idx >= total) return;
-  const int blk16 = static_cast<int>(idx % bpr);
-  int64_t r = idx / bpr;
-  const int h = static_cast<int>(r % p.H);
-  r /= p.H;
-  const int kv = static_cast<int>(r & 1);
-  const int64_t t = r >> 1;
-  const float g = __ldg(kv ? p.v_scale : p.k_scale);
-  if (!(g >= 0.f && g < kInf)) {
-    if (idx == 0 || idx == bpr * p.H) set_err(p.d_err, kErrScale);
-    return;
-  }
-  const int64_t slot = resolve_slot(p, t);
-  if (slot < 0) return;
-  const uint16_t* src = (kv ? p.v : p.k) + (t * p.H + h) * p.D + 16 * blk16;
-  const uint4 x0 = __ldg(reinterpret_cast<const uint4*>(src));
-  const uint4 x1 = __ldg(reinterpret_cast<const uint4*>(src) + 1);
-  const uint32_t w[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-  float v[16];
-  float bmax = 0.f;
+  const int lg = p.D == 128 ? 4 : 3, per_kv = p.H << lg, n = 2 * per_kv, total = tpb * n;
+  const float ks = __ldg(p.k_scale), vs = __ldg(p.v_scale);
+  const bool ok_k = ks > 0.f && ks < kInf, ok_v = vs > 0.f && vs < kInf;
+  if (blockIdx.x == 0 && threadIdx.x == 0 && !(ok_k && ok_v)) set_err(p.d_err, kErrScale);
+  __shared__ TokSlots ts;
+  for (int64_t t0 = static_cast<int64_t>(blockIdx.x) * tpb; t0 < p.T;
+       t0 += static_cast<int64_t>(gridDim.x) * tpb) {
+    block_slots(p, t0, tpb, ts);
+    for (int ii0 = threadIdx.x; ii0 < total; ii0 += kBatch * blockDim.x) {
+      uint4 x[kBatch];
+      uint8_t* dst[kBatch];
+      float sc[kBatch];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    v[2 * i] = bf16_lo(w[i]);
-    v[2 * i + 1] = bf16_hi(w[i]);
-    bmax = fmaxf(bmax, fmaxf(fabsf(v[2 * i]), fabsf(v[2 * i + 1])));
-  }
-  uint32_t sb = 0, codes_lo = 0, codes_hi = 0;
-  if (g > 0.f) {
-    sb = f32x2_to_e4m3x2(__fdiv_rn(bmax, __fmul_rn(6.0f, g)), 0.f) & 0xFFu;
-    const float den = __fmul_rn(e4m3_to_f32(sb), g);
-    if (den != 0.f) {
+      for (int u = 0; u < kBatch; ++u) {
+        dst[u] = nullptr;
+        const int ii = ii0 + u * blockDim.x;
+        if (ii >= total) continue;
+        const Chunk q = chunk_of(ts, t0, ii, n, per_kv, lg);
+        if (q.slot < 0 || !(q.kv ? ok_v : ok_k)) continue;
+        sc[u] = q.kv ? vs : ks;
+        x[u] = __ldg(reinterpret_cast<const uint4*>((q.kv ? p.v : p.k) +
+                                                    (q.t * p.H + q.h) * p.D + 8 * q.c));
+        dst[u] = (q.kv ? p.vc : p.kc) +
+                 ((q.slot / kPage * p.H + q.h) * kPage + q.slot % kPage) * p.D + 8 * q.c;
+      }
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        codes_lo |= f32x2_to_e2m1x2(__fdiv_rn(v[2 * i], den), __fdiv_rn(v[2 * i + 1], den))
-                    << (8 * i);
-        codes_hi |= f32x2_to_e2m1x2(__fdiv_rn(v[8 + 2 * i], den), __fdiv_rn(v[9 + 2 * i], den))
-                    << (8 * i);
+      for (int u = 0; u < kBatch; ++u) {
+        if (!dst[u]) continue;
+        const uint32_t w[4] = {x[u].x, x[u].y, x[u].z, x[u].w};
+        uint32_t code[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          code[e] = f32x2_to_e4m3x2(__fdiv_rn(bf16_lo(w[e]), sc[u]),
+                                    __fdiv_rn(bf16_hi(w[e]), sc[u]));
+        *reinterpret_cast<uint2*>(dst[u]) =
+            make_uint2(code[0] | (code[1] << 16), code[2] | (code[3] << 16));
       }
     }
+    __syncthreads();  // ts is rewritten for the next tokens
   }
-  uint8_t* page = (kv ? p.vc : p.kc) + (slot / kPage * p.H + h) * static_cast<int64_t>(9 * p.D);
-  const int o = static_cast<int>(slot % kPage);
-  *reinterpret_cast<uint2*>(page + o * (p.D / 2) + 8 * blk16) = make_uint2(codes_lo, codes_hi);
-  page[8 * p.D + o * (p.D / 16) + blk16] = static_cast<uint8_t>(sb);
 }
 
-// One thread = 8 elements (16 bytes) of one (token, K|V, head) row.
-__global__ void write_bf16_kernel(const QuantParams p) {
+// One chunk = one 16-element block of one (K|V, head) row of a token.
+__global__ void quantize_nvfp4_kernel(const QuantParams p, int tpb) {
   griddep_launch_dependents();  // a following decode may start its prologue
-  const int cpr = p.D / 8;
-  const int64_t total = p.T * 2 * p.H * cpr;
-  const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (idx >= total) return;
-  const int c = static_cast<int>(idx % cpr);
-  int64_t r = idx / cpr;
-  const int h = static_cast<int>(r % p.H);
-  r /= p.H;
-  const int kv = static_cast<int>(r & 1);
-  const int64_t t = r >> 1;
-  const int64_t slot = resolve_slot(p, t);
-  if (slot < 0) return;
-  const uint16_t* src = (kv ? p.v : p.k) + (t * p.H + h) * p.D + 8 * c;
-  uint8_t* dst = (kv ? p.vc : p.kc) +
-                 (((slot / kPage * p.H + h) * kPage + slot % kPage) * p.D + 8 * c) * 2;
-  *reinterpret_cast<uint4*>(dst) = __ldg(reinterpret_cast<const uint4*>(src));
+  const int lg = p.D == 128 ? 3 : 2, per_kv = p.H << lg, n = 2 * per_kv, total = tpb * n;
+  const float gk = __ldg(p.k_scale), gv = __ldg(p.v_scale);
+  const bool ok_k = gk >= 0.f && gk < kInf, ok_v = gv >= 0.f && gv < kInf;
+  if (blockIdx.x == 0 && threadIdx.x == 0 && !(ok_k && ok_v)) set_err(p.d_err, kErrScale);
+  __shared__ TokSlots ts;
+  for (int64_t t0 = static_cast<int64_t>(blockIdx.x) * tpb; t0 < p.T;
+       t0 += static_cast<int64_t>(gridDim.x) * tpb) {
+    block_slots(p, t0, tpb, ts);
+    for (int ii0 = threadIdx.x; ii0 < total; ii0 += kBatchNv * blockDim.x) {
+      uint4 x0[kBatchNv], x1[kBatchNv];
+      uint8_t* page[kBatchNv];
+      float gg[kBatchNv];
+      int o[kBatchNv], blk16[kBatchNv];
+#pragma unroll
+      for (int u = 0; u < kBatchNv; ++u) {
+        page[u] = nullptr;
+        const int ii = ii0 + u * blockDim.x;
+        if (ii >= total) continue;
+        const Chunk q = chunk_of(ts, t0, ii, n, per_kv, lg);
+        if (q.slot < 0 || !(q.kv ? ok_v : ok_k)) continue;
+        gg[u] = q.kv ? gv : gk;
+        const uint4* src = reinterpret_cast<const uint4*>((q.kv ? p.v : p.k) +
+                                                          (q.t * p.H + q.h) * p.D + 16 * q.c);
+        x0[u] = __ldg(src);
+        x1[u] = __ldg(src + 1);
+        page[u] = (q.kv ? p.vc : p.kc) +
+                  (q.slot / kPage * p.H + q.h) * static_cast<int64_t>(9 * p.D);
+        o[u] = static_cast<int>(q.slot % kPage);
+        blk16[u] = q.c;
+      }
+#pragma unroll
+      for (int u = 0; u < kBatchNv; ++u) {
+        if (!page[u]) continue;
+        const float g = gg[u];
+        const uint32_t w[8] = {x0[u].x, x0[u].y, x0[u].z, x0[u].w,
+                               x1[u].x, x1[u].y, x1[u].z, x1[u].w};
+        float v[16];
+        float bmax = 0.f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          v[2 * e] = bf16_lo(w[e]);
+          v[2 * e + 1] = bf16_hi(w[e]);
+          bmax = fmaxf(bmax, fmaxf(fabsf(v[2 * e]), fabsf(v[2 * e + 1])));
+        }
+        uint32_t sb = 0, codes_lo = 0, codes_hi = 0;
+        if (g > 0.f) {
+          sb = f32x2_to_e4m3x2(__fdiv_rn(bmax, __fmul_rn(6.0f, g)), 0.f) & 0xFFu;
+          const float den = __fmul_rn(e4m3_to_f32(sb), g);
+          if (den != 0.f) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              codes_lo |= f32x2_to_e2m1x2(__fdiv_rn(v[2 * e], den),
+                                          __fdiv_rn(v[2 * e + 1], den))
+                          << (8 * e);
+              codes_hi |= f32x2_to_e2m1x2(__fdiv_rn(v[8 + 2 * e], den),
+                                          __fdiv_rn(v[9 + 2 * e], den))
+                          << (8 * e);
+            }
+          }
+        }
+        *reinterpret_cast<uint2*>(page[u] + o[u] * (p.D / 2) + 8 * blk16[u]) =
+            make_uint2(codes_lo, codes_hi);
+        page[u][8 * p.D + o[u] * (p.D / 16) + blk16[u]] = static_cast<uint8_t>(sb);
+      }
+    }
+    __syncthreads();  // ts is rewritten for the next tokens
+  }
+}
+
+// One chunk = 8 elements (16 bytes) of one (K|V, head) row of a token.
+__global__ void write_bf16_kernel(const QuantParams p, int tpb) {
+  griddep_launch_dependents();  // a following decode may start its prologue
+  const int lg = p.D == 128 ? 4 : 3, per_kv = p.H << lg, n = 2 * per_kv, total = tpb * n;
+  __shared__ TokSlots ts;
+  for (int64_t t0 = static_cast<int64_t>(blockIdx.x) * tpb; t0 < p.T;
+       t0 += static_cast<int64_t>(gridDim.x) * tpb) {
+    block_slots(p, t0, tpb, ts);
+    for (int ii0 = threadIdx.x; ii0 < total; ii0 += kBatch * blockDim.x) {
+      uint4 x[kBatch];
+      uint8_t* dst[kBatch];
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        dst[u] = nullptr;
+        const int ii = ii0 + u * blockDim.x;
+        if (ii >= total) continue;
+        const Chunk q = chunk_of(ts, t0, ii, n, per_kv, lg);
+        if (q.slot < 0) continue;
+        x[u] = __ldg(reinterpret_cast<const uint4*>((q.kv ? p.v : p.k) +
+                                                    (q.t * p.H + q.h) * p.D + 8 * q.c));
+        dst[u] = (q.kv ? p.vc : p.kc) +
+                 (((q.slot / kPage * p.H + q.h) * kPage + q.slot % kPage) * p.D + 8 * q.c) * 2;
+      }
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u)
+        if (dst[u]) *reinterpret_cast<uint4*>(dst[u]) = x[u];
+    }
+    __syncthreads();  // ts is rewritten for the next tokens
+  }
 }
 
 // One thread = 8 elements of one (slot, K|V, head) row.
@@ -274,13 +355,19 @@ unsigned grid_for(int64_t total, int threads) {
 
 cudaError_t launch_quantize(int fmt, const QuantParams& p, cudaStream_t stream) {
   if (p.T == 0) return cudaSuccess;
+  // Tokens per block: as many as keep >= 4 blocks per SM (so a short write
+  // stays spread over SMs, a long one pays one slot lookup chain per block).
   const int threads = 256;
+  int tpb = 1;
+  while (tpb < kTokPerBlock && p.T / (2 * tpb) >= 4 * static_cast<int64_t>(num_sms())) tpb *= 2;
+  const int64_t blocks = (p.T + tpb - 1) / tpb;
+  const unsigned grid = static_cast<unsigned>(blocks < (1 << 20) ? blocks : (1 << 20));
   if (fmt == 1) {
-    quantize_fp8_kernel<<<grid_for(p.T * 2 * p.H * (p.D / 8), threads), threads, 0, stream>>>(p);
+    quantize_fp8_kernel<<<grid, threads, 0, stream>>>(p, tpb);
   } else if (fmt == 2) {
-    quantize_nvfp4_kernel<<<grid_for(p.T * 2 * p.H * (p.D / 16), threads), threads, 0, stream>>>(p);
+    quantize_nvfp4_kernel<<<grid, threads, 0, stream>>>(p, tpb);
   } else {
-    write_bf16_kernel<<<grid_for(p.T * 2 * p.H * (p.D / 8), threads), threads, 0, stream>>>(p);
+    write_bf16_kernel<<<grid, threads, 0, stream>>>(p, tpb);
   }
   return cudaGetLastError();
 }
