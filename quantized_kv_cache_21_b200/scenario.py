@@ -104,8 +104,9 @@ class DecodeScenario:
     def scan_bytes(self) -> int:
         return kv_scan_bytes(self.fmt, self.lens, self.H, self.D)
 
-    def write(self, stream=None):
-        kvq.kv_quantize_write(self.fmt, self.step_k, self.step_v, self.step_slots, self.cache,
+    def write(self, stream=None, k=None, v=None):
+        kvq.kv_quantize_write(self.fmt, self.step_k if k is None else k,
+                              self.step_v if v is None else v, self.step_slots, self.cache,
                               self.d_ks, self.d_vs, self.err, block_table=self.d_bt,
                               stream=stream)
 
