@@ -841,25 +841,30 @@ __global__ void __launch_bounds__(Shape<FMT, D>::NW * 32, 1)
     }
   }
 
-  // Issue the copies of local item i into stage i % NSW (all lanes call;
-  // lane 0 issues).  stage_ok (warp-uniform) records which stages hold a
-  // valid page; a bad block id completes its stage's phase with no data.
+  // Issue the copies of local item i into stage stg (= i % NSW; all lanes
+  // call).  The lane holding item i's block id in the window issues them, so
+  // no shuffle is needed; ok_win (one ballot per window) says which items of
+  // the window have a valid block id.  stage_ok (warp-uniform) records which
+  // stages hold a valid page; a bad block id completes its stage's phase with
+  // no data.
+  unsigned ok_win = __ballot_sync(0xffffffffu, cur_blk >= 0 && cur_blk < p.num_blocks);
   unsigned stage_ok = 0;
-  auto issue = [&](int i) {
+  auto issue = [&](int i, int stg) {
     if (i >= chunk + 32) {  // slide the id window by 32 items
       chunk += 32;
       cur_blk = nxt_blk;
       cur_h = nxt_h;
       item_block(p, tab, u0, vbeg, vend, warp + (chunk + 32 + lane) * NW, nxt_blk, nxt_h);
+      ok_win = __ballot_sync(0xffffffffu, cur_blk >= 0 && cur_blk < p.num_blocks);
     }
-    const int blk = __shfl_sync(0xffffffffu, cur_blk, i - chunk);
-    const int h = __shfl_sync(0xffffffffu, cur_h, i - chunk);
-    const bool ok = blk >= 0 && blk < p.num_blocks;
-    stage_ok = (stage_ok & ~(1u << (i % NSW))) | (static_cast<unsigned>(ok) << (i % NSW));
-    if (lane == 0) {
-      uint64_t* bar = &bars[i % NSW];
+    const int src = i - chunk;
+    const unsigned ok = (ok_win >> src) & 1u;
+    stage_ok = (stage_ok & ~(1u << stg)) | (ok << stg);
+    if (lane == src) {
+      uint64_t* bar = &bars[stg];
+      fence_proxy_async_smem();  // the warp's reads of this stage precede the copy
       if (ok) {
-        F::issue(ring + (i % NSW) * F::STAGE, bar, &mk, &mv, &mks, &mvs, h, blk);
+        F::issue(ring + stg * F::STAGE, bar, &mk, &mv, &mks, &mvs, cur_h, cur_blk);
       } else {
         set_err(p.d_err, kErrBlockId);
         mbar_arrive(bar);  // completes the phase with no data; the page is skipped
@@ -869,12 +874,11 @@ __global__ void __launch_bounds__(Shape<FMT, D>::NW * 32, 1)
   // Prologue: lane i fills stage i with local item i (its own cur_blk), the
   // lanes' copies issued together rather than one after another.
   {
-    const bool ok = cur_blk >= 0 && cur_blk < p.num_blocks;
     const int n0 = min(NSW, n_local);
-    stage_ok = __ballot_sync(0xffffffffu, ok) & ((1u << n0) - 1u);
+    stage_ok = ok_win & ((1u << n0) - 1u);
     if (lane < n0) {
       uint64_t* bar = &bars[lane];
-      if (ok) {
+      if ((ok_win >> lane) & 1u) {
         F::issue(ring + lane * F::STAGE, bar, &mk, &mv, &mks, &mvs, cur_h, cur_blk);
       } else {
         set_err(p.d_err, kErrBlockId);
@@ -885,6 +889,7 @@ __global__ void __launch_bounds__(Shape<FMT, D>::NW * 32, 1)
 
   const float c_log2 = p.sm_scale * ks * kLog2e;
   int k_base = 0, j = 0;  // j = this warp's next local item
+  int st = 0, ph = 0;     // its stage (j % NSW) and barrier phase parity ((j / NSW) & 1)
   for (int si = 0; si < nu; ++si) {
     const int u = u0 + si;
     const int grp = u % p.n_groups, h = (u / p.n_groups) % p.Hkv, b = u / (p.n_groups * p.Hkv);
@@ -913,10 +918,9 @@ __global__ void __launch_bounds__(Shape<FMT, D>::NW * 32, 1)
 
     const int k_end = k_base + n_items;
     for (int k = warp + j * NW; k < k_end; k += NW, ++j) {
-      const int st = j % NSW;
       const uint8_t* sp = ring + st * F::STAGE;
       // all lanes agree on the outcome so the warp stays converged
-      if (!__all_sync(0xffffffffu, mbar_wait_bounded(&bars[st], (j / NSW) & 1))) {
+      if (!__all_sync(0xffffffffu, mbar_wait_bounded(&bars[st], ph))) {
         if (lane == 0) set_err(p.d_err, kErrTimeout);
         for (int i = j + 1; i < j + NSW && i < n_local; ++i)  // drain copies in flight
           mbar_wait_bounded(&bars[i % NSW], (i / NSW) & 1);
@@ -954,9 +958,10 @@ __global__ void __launch_bounds__(Shape<FMT, D>::NW * 32, 1)
         F::load_raw(sp, gid, tig, raw);
       }
       __syncwarp();
-      if (j + NSW < n_local) {
-        if (lane == 0) fence_proxy_async_smem();
-        issue(j + NSW);
+      if (j + NSW < n_local) issue(j + NSW, st);  // item j + NSW reuses stage st
+      if (++st == NSW) {
+        st = 0;
+        ph ^= 1;
       }
       if (!valid) continue;
       if constexpr (!F::kLateV) qk();
