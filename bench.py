@@ -51,6 +51,11 @@ def parse():
     ap.add_argument("--workload", default=MAIN_WORKLOAD)
     ap.add_argument("--no-extras", action="store_true", help="main line only")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--sweep", action="store_true",
+                    help="instead of the bench line: decode time of every sweep cell "
+                         "(context x batch x head_dim x format), one JSON line each")
+    ap.add_argument("--sweep-formats", default="bf16,fp8,nvfp4")
+    ap.add_argument("--sweep-dims", default="64,128")
     return ap.parse_args()
 
 
@@ -274,10 +279,63 @@ def roofline(bytes_per_launch, ms_list, peak, peak_kind, traffic):
             "kernel": "kvq_decode_kernel", "us_per_launch": ms * 1e3}
 
 
+def run_sweep(args):
+    """Decode-only timing of the sweep cells on one GPU (L2 flushed before every
+    timed launch).  Prints one JSON line per cell, then a summary line."""
+    import dataclasses
+    import torch
+    import quantized_kv_cache_21_b200 as kvq
+    from quantized_kv_cache_21_b200 import workloads as wl
+    from quantized_kv_cache_21_b200.scenario import DecodeScenario
+
+    kvq.lib()
+    clocks = ClockSampler(torch.cuda.current_device())
+    timer = Timer(torch, clocks)
+    peak, peak_kind = measured_hbm_peak()
+    K, W = max(3, args.steps), max(3, args.warmup)
+    cells = []
+    for D in (int(x) for x in args.sweep_dims.split(",")):
+        for fmt in args.sweep_formats.split(","):
+            for L in wl.SWEEP_LENGTHS:
+                for B in wl.SWEEP_BATCHES:
+                    w = dataclasses.replace(wl.SWEEP, B=B, D=D, seq_len=L)
+                    lens = wl.varlen(wl.rng_for(wl.SWEEP_SEED, wl.sweep_cell_stream(L, B)), B, L)
+                    sc = DecodeScenario(w, fmt=fmt, lens=lens)
+                    (dms,), _ = timer.run([sc.decode], K, W)
+                    assert int(sc.err.item()) == 0
+                    us = statistics.median(dms) * 1e3
+                    gbps = sc.scan_bytes / (us * 1e-6) / 1e9
+                    cell = {"sweep_cell": {"format": fmt, "head_dim": D, "context": L, "batch": B,
+                                           "kv_heads": 8, "q_heads": 64,
+                                           "lengths": "uniform in [L/2, L]"},
+                            "kv_scan_bytes": sc.scan_bytes, "us_per_decode": us, "GBps": gbps,
+                            "frac_of_hbm_peak": gbps / peak}
+                    print(json.dumps(cell), flush=True)
+                    cells.append(cell)
+                    del sc
+                    torch.cuda.empty_cache()
+    heavy = [c for c in cells if c["kv_scan_bytes"] >= 64e6]
+    summary = {"sweep_summary": {
+        "cells": len(cells), "peak_GBps": peak, "peak_source": peak_kind,
+        "byte_heavy_cells (>= 64 MB)": len(heavy),
+        "min_frac_byte_heavy": {f: min((c["frac_of_hbm_peak"] for c in heavy
+                                        if c["sweep_cell"]["format"] == f), default=None)
+                                for f in args.sweep_formats.split(",")},
+        "median_frac_byte_heavy": {f: statistics.median([c["frac_of_hbm_peak"] for c in heavy
+                                                         if c["sweep_cell"]["format"] == f])
+                                   if any(c["sweep_cell"]["format"] == f for c in heavy)
+                                   else None for f in args.sweep_formats.split(",")},
+        "clocks": clocks.summary()}}
+    print(json.dumps(summary))
+    return 0
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         return run_reference(args)
+    if args.sweep:
+        return run_sweep(args)
     import torch
     import quantized_kv_cache_21_b200 as kvq
     from quantized_kv_cache_21_b200 import workloads as wl

@@ -26,7 +26,9 @@ def kv_scan_bytes(fmt: str, lens, H: int, D: int) -> int:
 
 class DecodeScenario:
     def __init__(self, w: wl.Workload, fmt: str | None = None, device: str = "cuda",
-                 seq_offset: int = 0):
+                 seq_offset: int = 0, lens=None):
+        """lens: optional per-sequence lengths (each in [chunk, seq_len]); by
+        default every sequence holds seq_len tokens."""
         self.w = w
         self.fmt = fmt or w.fmt
         self.device = device
@@ -38,7 +40,9 @@ class DecodeScenario:
         rng = wl.rng_for(w.seed, 1)
         self.bt = (wl.permuted_block_table(rng, B, self.mb) if w.permuted
                    else wl.identity_block_table(B, self.mb))
-        self.lens = np.full(B, L, np.int32)
+        self.lens = (np.full(B, L, np.int32) if lens is None
+                     else np.asarray(lens, dtype=np.int32).reshape(B))
+        assert self.lens.max(initial=0) <= L and self.lens.min(initial=L) >= self.chunk
         self.out_k = wl.outliers_for(w, H, D, "k")
         self.out_v = wl.outliers_for(w, H, D, "v")
         self.seq_offset = seq_offset  # a rank's sequences draw distinct sub-streams
@@ -56,7 +60,7 @@ class DecodeScenario:
         if self.fmt != "bf16":
             for b in range(B if w.calib_tokens is None else 1):
                 k, v = self.tokens(b)
-                n = L if w.calib_tokens is None else w.calib_tokens
+                n = int(self.lens[b]) if w.calib_tokens is None else w.calib_tokens
                 kvq.kv_calibrate_absmax(k[:n].contiguous(), self.amax[0:1])
                 kvq.kv_calibrate_absmax(v[:n].contiguous(), self.amax[1:2])
                 del k, v
@@ -65,21 +69,23 @@ class DecodeScenario:
 
         # fill the context (all but the step's chunk), keep the chunk for the step
         step_k, step_v = [], []
-        ctx = L - self.chunk
         for b in range(B):
             k, v = self.tokens(b)
+            n = int(self.lens[b])
+            ctx = n - self.chunk
             if ctx > 0:
                 slots = torch.from_numpy(wl.physical_slots(self.bt, b, np.arange(ctx))).to(dev)
                 kvq.kv_quantize_write(self.fmt, k[:ctx], v[:ctx], slots, self.cache, self.d_ks,
                                       self.d_vs, self.err)
-            step_k.append(k[ctx:].clone())
-            step_v.append(v[ctx:].clone())
+            step_k.append(k[ctx:n].clone())
+            step_v.append(v[ctx:n].clone())
             del k, v
         self.step_k = torch.cat(step_k).contiguous()
         self.step_v = torch.cat(step_v).contiguous()
         # logical slots (seq * max_blocks * 16 + position) of the step's tokens,
         # translated through the block table inside the write kernel
-        logical = np.concatenate([b * self.mb * wl.PAGE + np.arange(ctx, L) for b in range(B)])
+        logical = np.concatenate([b * self.mb * wl.PAGE + np.arange(int(n) - self.chunk, int(n))
+                                  for b, n in enumerate(self.lens)])
         self.step_slots = torch.from_numpy(logical.astype(np.int64)).to(dev)
 
         g = torch.Generator(device=dev)

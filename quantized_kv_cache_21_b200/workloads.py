@@ -126,6 +126,22 @@ WORKLOADS = {
                                   {"frac": 0.01}, {"frac": 0.01}, 16.0, 16384, True, 2048),
 }
 
+# The sweep: context L in 1k/4k/16k/64k/128k tokens x batch 1/8/32/64, lengths
+# uniform in [L/2, L] (varlen), GQA 8 (8 KV heads, 64 query heads), head_dim
+# 64 and 128, BF16/FP8/NVFP4; plain N(0,1) K/V.  One cell = this template with
+# B, D and seq_len set, and per-sequence lengths drawn with
+# varlen(rng_for(SWEEP_SEED, sweep_cell_stream(L, B)), B, L).
+SWEEP_LENGTHS = (1024, 4096, 16384, 65536, 131072)
+SWEEP_BATCHES = (1, 8, 32, 64)
+SWEEP_SEED = 20264
+SWEEP = Workload("sweep", "fp8", 1, 8, 64, 128, 1024, SWEEP_SEED)
+
+
+def sweep_cell_stream(L: int, B: int) -> int:
+    """Sub-stream of a sweep cell's length draw (same lengths for every format
+    and head_dim)."""
+    return 1000 + 10 * SWEEP_LENGTHS.index(L) + SWEEP_BATCHES.index(B)
+
 
 def device_tokens(seed: int, stream: int, T: int, H: int, D: int,
                   outliers: list[tuple[int, int]] = (), factor: float = 1.0,
