@@ -52,6 +52,9 @@ namespace {
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kPScale = 4096.0f;  // P is fed to the MMA as p * 2^12 (exact)
+// A warp's running max lags the true max by < kRescaleGap (log2 units), so
+// p <= 2^3 and p * kPScale <= 2^15 < 65504, the largest f16.
+constexpr float kRescaleGap = 3.0f;
 
 // --------------------------------------------------------------------------
 // Per-(format, head_dim) fragment layouts.
@@ -912,6 +915,7 @@ __global__ void __launch_bounds__(Shape<FMT, D>::NW * 32, 1)
     if (si > 0) load_q(u);
 
     float m0 = -kInf, m1 = -kInf, l0 = 0.f, l1 = 0.f;
+    float t0 = -kInf, t1 = -kInf;  // rescale thresholds m + kRescaleGap
     float o[MT][4];
 #pragma unroll
     for (int jj = 0; jj < MT; ++jj) o[jj][0] = o[jj][1] = o[jj][2] = o[jj][3] = 0.f;
@@ -985,16 +989,19 @@ __global__ void __launch_bounds__(Shape<FMT, D>::NW * 32, 1)
         }
       }
 
-      // ---- online softmax (log2 domain); this thread: heads 2tig, 2tig+1
-      float mx0 = fmaxf(s0, s2), mx1 = fmaxf(s1, s3);
+      // ---- online softmax (log2 domain); this thread: heads 2tig, 2tig+1.
+      // The running max m moves only when a score passes m + kRescaleGap
+      // (one vote, no reduction, on most pages); p = 2^(s - m) then stays
+      // <= 2^kRescaleGap, which keeps p * kPScale inside f16.
+      if (__any_sync(0xffffffffu, s0 > t0 || s2 > t0 || s1 > t1 || s3 > t1)) {
+        float mx0 = fmaxf(s0, s2), mx1 = fmaxf(s1, s3);
 #pragma unroll
-      for (int off = 4; off < 32; off <<= 1) {
-        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
-        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
-      }
-      const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
-      if (__any_sync(0xffffffffu, mn0 != m0 || mn1 != m1)) {
-        const float a0 = fast_exp2(m0 - mn0), a1 = fast_exp2(m1 - mn1);
+        for (int off = 4; off < 32; off <<= 1) {
+          mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+          mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+        }
+        const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
+        const float a0 = fast_exp2(m0 - mn0), a1 = fast_exp2(m1 - mn1);  // 0 while m = -inf
         l0 *= a0;
         l1 *= a1;
 #pragma unroll
@@ -1006,6 +1013,8 @@ __global__ void __launch_bounds__(Shape<FMT, D>::NW * 32, 1)
         }
         m0 = mn0;
         m1 = mn1;
+        t0 = m0 + kRescaleGap;
+        t1 = m1 + kRescaleGap;
       }
       const float p0 = fast_exp2(s0 - m0), p1 = fast_exp2(s1 - m1);
       const float p2 = fast_exp2(s2 - m0), p3 = fast_exp2(s3 - m1);
