@@ -51,10 +51,14 @@ namespace {
 
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr float kPScale = 4096.0f;  // P is fed to the MMA as p * 2^12 (exact)
-// A warp's running max lags the true max by < kRescaleGap (log2 units), so
-// p <= 2^3 and p * kPScale <= 2^15 < 65504, the largest f16.
+// P is fed to the MMA as p * 2^kPLog2 (computed directly as 2^(s - m + 12)),
+// so small probabilities stay clear of the f16 subnormals; l and O carry the
+// same factor.  A warp's running max m lags the true max by at most
+// kRescaleGap (log2 units): p <= 2^3, P <= 2^15 < 65504, the largest f16.
+constexpr float kPLog2 = 12.0f;
+constexpr float kPScale = 4096.0f;  // 2^kPLog2
 constexpr float kRescaleGap = 3.0f;
+constexpr float kETop = kPLog2 + kRescaleGap;  // e = s - m + kPLog2 above this moves m
 
 // --------------------------------------------------------------------------
 // Per-(format, head_dim) fragment layouts.
@@ -680,11 +684,11 @@ __device__ __forceinline__ void final_merge(const DecodeParams& p, int u, int b,
       }
       M = Mn;
     }
-    const float sc = L > 0.f ? vs / (L * kPScale) : 0.f;
+    const float sc = L > 0.f ? vs / L : 0.f;
     const size_t row = static_cast<size_t>(b) * p.Hq + h * p.G + qi;
     *reinterpret_cast<float4*>(p.out + row * D + d4) =
         make_float4(acc.x * sc, acc.y * sc, acc.z * sc, acc.w * sc);
-    if (d4 == 0 && p.lse) p.lse[row] = L > 0.f ? (M + log2f(L)) * kLn2 : -kInf;
+    if (d4 == 0 && p.lse) p.lse[row] = L > 0.f ? (M + log2f(L) - kPLog2) * kLn2 : -kInf;
   }
 }
 
@@ -915,12 +919,14 @@ __global__ void __launch_bounds__(Shape<FMT, D>::NW * 32, 1)
     if (si > 0) load_q(u);
 
     float m0 = -kInf, m1 = -kInf, l0 = 0.f, l1 = 0.f;
-    float t0 = -kInf, t1 = -kInf;  // rescale thresholds m + kRescaleGap
+    float n0 = kInf, n1 = kInf;  // kPLog2 - m
     float o[MT][4];
 #pragma unroll
     for (int jj = 0; jj < MT; ++jj) o[jj][0] = o[jj][1] = o[jj][2] = o[jj][3] = 0.f;
 
     const int k_end = k_base + n_items;
+    // valid tokens of the segment's last page (only that page can be partial)
+    const int n_last = len - (ps + n_items - 1) * kPage;
     for (int k = warp + j * NW; k < k_end; k += NW, ++j) {
       const uint8_t* sp = ring + st * F::STAGE;
       // all lanes agree on the outcome so the warp stays converged
@@ -931,8 +937,6 @@ __global__ void __launch_bounds__(Shape<FMT, D>::NW * 32, 1)
         j = n_local;
         break;
       }
-      const int page = ps + (k - k_base);
-      const int n_valid = min(kPage, len - page * kPage);
       const bool valid = (stage_ok >> st) & 1u;
 
       // The stage's words go to registers first, so the stage is refilled with
@@ -971,11 +975,12 @@ __global__ void __launch_bounds__(Shape<FMT, D>::NW * 32, 1)
       if constexpr (!F::kLateV) qk();
       F::conv_v(raw, va);
 
-      float s0 = (sa[0] + sb[0]) * c_log2, s1 = (sa[1] + sb[1]) * c_log2;
-      float s2 = (sa[2] + sb[2]) * c_log2, s3 = (sa[3] + sb[3]) * c_log2;
-      if (n_valid < kPage) {  // last, partial page: mask tokens past the length
-        if (gid >= n_valid) s0 = s1 = -kInf;
-        if (gid + 8 >= n_valid) s2 = s3 = -kInf;
+      // raw scores r = q . k_code (the scale c_log2 is applied below)
+      float r0 = sa[0] + sb[0], r1 = sa[1] + sb[1], r2 = sa[2] + sb[2], r3 = sa[3] + sb[3];
+      if (k == k_end - 1 && n_last < kPage) {  // last, partial page: mask tokens past the length
+        const int n_valid = n_last;
+        if (gid >= n_valid) r0 = r1 = -kInf;
+        if (gid + 8 >= n_valid) r2 = r3 = -kInf;
         const uint32_t m01 = (2 * tig < n_valid ? 0x0000FFFFu : 0u) |
                              (2 * tig + 1 < n_valid ? 0xFFFF0000u : 0u);
         const uint32_t m23 = (2 * tig + 8 < n_valid ? 0x0000FFFFu : 0u) |
@@ -992,8 +997,12 @@ __global__ void __launch_bounds__(Shape<FMT, D>::NW * 32, 1)
       // ---- online softmax (log2 domain); this thread: heads 2tig, 2tig+1.
       // The running max m moves only when a score passes m + kRescaleGap
       // (one vote, no reduction, on most pages); p = 2^(s - m) then stays
-      // <= 2^kRescaleGap, which keeps p * kPScale inside f16.
-      if (__any_sync(0xffffffffu, s0 > t0 || s2 > t0 || s1 > t1 || s3 > t1)) {
+      // <= 2^kRescaleGap, which keeps P = p * 2^kPLog2 inside f16.
+      // e = s - m + kPLog2 with s = c_log2 * r: 2^e = p * 2^kPLog2 = P as fed to the MMA
+      float e0 = fmaf(r0, c_log2, n0), e1 = fmaf(r1, c_log2, n1);
+      float e2 = fmaf(r2, c_log2, n0), e3 = fmaf(r3, c_log2, n1);
+      if (__any_sync(0xffffffffu, e0 > kETop || e2 > kETop || e1 > kETop || e3 > kETop)) {
+        const float s0 = r0 * c_log2, s1 = r1 * c_log2, s2 = r2 * c_log2, s3 = r3 * c_log2;
         float mx0 = fmaxf(s0, s2), mx1 = fmaxf(s1, s3);
 #pragma unroll
         for (int off = 4; off < 32; off <<= 1) {
@@ -1013,32 +1022,34 @@ __global__ void __launch_bounds__(Shape<FMT, D>::NW * 32, 1)
         }
         m0 = mn0;
         m1 = mn1;
-        t0 = m0 + kRescaleGap;
-        t1 = m1 + kRescaleGap;
+        n0 = kPLog2 - m0;
+        n1 = kPLog2 - m1;
+        e0 = s0 + n0;
+        e1 = s1 + n1;
+        e2 = s2 + n0;
+        e3 = s3 + n1;
       }
-      const float p0 = fast_exp2(s0 - m0), p1 = fast_exp2(s1 - m1);
-      const float p2 = fast_exp2(s2 - m0), p3 = fast_exp2(s3 - m1);
-      l0 += p0 + p2;
-      l1 += p1 + p3;
+      const float q0 = fast_exp2(e0), q1 = fast_exp2(e1), q2 = fast_exp2(e2), q3 = fast_exp2(e3);
+      l0 += q0 + q2;  // l and O carry the factor 2^kPLog2, removed at normalisation
+      l1 += q1 + q3;
 
       // ---- P^T fragments: high part + residual, transposed in registers
-      const float q0 = p0 * kPScale, q1 = p1 * kPScale, q2 = p2 * kPScale, q3 = p3 * kPScale;
       uint32_t x0h, x1h, x0l, x1l;
-      float r0, r1, r2, r3;
+      float h0, h1, h2, h3;  // the high parts as fp32
       if constexpr (F::kBF16) {
         x0h = pack_bf16x2(q0, q1);
         x1h = pack_bf16x2(q2, q3);
-        unpack_bf16x2(x0h, r0, r1);
-        unpack_bf16x2(x1h, r2, r3);
-        x0l = pack_bf16x2(q0 - r0, q1 - r1);
-        x1l = pack_bf16x2(q2 - r2, q3 - r3);
+        unpack_bf16x2(x0h, h0, h1);
+        unpack_bf16x2(x1h, h2, h3);
+        x0l = pack_bf16x2(q0 - h0, q1 - h1);
+        x1l = pack_bf16x2(q2 - h2, q3 - h3);
       } else {
         x0h = pack_f16x2(q0, q1);
         x1h = pack_f16x2(q2, q3);
-        unpack_f16x2(x0h, r0, r1);
-        unpack_f16x2(x1h, r2, r3);
-        x0l = pack_f16x2(q0 - r0, q1 - r1);
-        x1l = pack_f16x2(q2 - r2, q3 - r3);
+        unpack_f16x2(x0h, h0, h1);
+        unpack_f16x2(x1h, h2, h3);
+        x0l = pack_f16x2(q0 - h0, q1 - h1);
+        x1l = pack_f16x2(q2 - h2, q3 - h3);
       }
       const uint32_t bh0 = movmatrix_t(x0h), bh1 = movmatrix_t(x1h);
       const uint32_t bl0 = movmatrix_t(x0l), bl1 = movmatrix_t(x1l);
@@ -1094,8 +1105,8 @@ __global__ void __launch_bounds__(Shape<FMT, D>::NW * 32, 1)
         const int qi = grp * 8 + hh;
         if (qi < p.G) {
           const size_t row = static_cast<size_t>(b) * p.Hq + h * p.G + qi;
-          p.out[row * D + d] = L > 0.f ? acc * (vs / (L * kPScale)) : 0.f;
-          if (d == 0 && p.lse) p.lse[row] = L > 0.f ? (M + log2f(L)) * kLn2 : -kInf;
+          p.out[row * D + d] = L > 0.f ? acc * (vs / L) : 0.f;
+          if (d == 0 && p.lse) p.lse[row] = L > 0.f ? (M + log2f(L) - kPLog2) * kLn2 : -kInf;
         }
       } else {
         gpart[16 + hh * D + d] = acc;
