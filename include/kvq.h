@@ -191,7 +191,16 @@ kvq_status kv_decode_workspace_size(int32_t fmt, int32_t num_seqs, int32_t num_q
  *                again, so it can be reused without clearing.  Calls that
  *                share a workspace must not overlap on the GPU.
  * Values are fp32-accumulated; results match float64 attention over the same
- * dequantised values to about 1e-4 absolute on out and 1e-6 relative on lse. */
+ * dequantised values to about 1e-4 absolute on out and 1e-6 relative on lse.
+ * Stream ordering: the launch allows programmatic dependent launch.  When the
+ * previous operation on the stream is a kv_quantize_write, the decode may
+ * start its prologue (reading q, block_table, seq_lens and the scales) while
+ * that write finishes, and waits for the write's cache stores before reading
+ * any cache page; those four inputs must therefore not be produced by that
+ * write's kernel (they never are).  After any other operation the launch is
+ * an ordinary stream-ordered one.  kv_quantize_write's kernels likewise let
+ * a following programmatic-dependent launch begin early: such a kernel must
+ * wait on its grid dependency before reading the cache. */
 kvq_status kv_decode_attention(int32_t fmt, const void* q, const kvq_cache* cache,
                                const int32_t* block_table, int32_t max_blocks,
                                const int32_t* seq_lens, int32_t num_seqs, int32_t num_q_heads,
