@@ -710,6 +710,8 @@ __global__ void __launch_bounds__(Shape<FMT, D>::NW * 32, 1)
   uint64_t* bars_all = reinterpret_cast<uint64_t*>(slots + NW * S::WPART);
   __shared__ UnitTable tab;
   __shared__ int s_last;  // this CTA completes the unit's cross-CTA merge
+  __shared__ float s_wt[NW][8];  // segment merge: warp weights per head
+  __shared__ float s_ml[2][8];   // segment merge: max and weighted sum per head
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int gid = lane >> 2, tig = lane & 3;
@@ -1085,22 +1087,31 @@ __global__ void __launch_bounds__(Shape<FMT, D>::NW * 32, 1)
       wp[16 + (2 * tig + 1) * D + d1] = o[jj][3];
     }
     __syncthreads();
+    // per head: the max M over the warps, each warp's weight 2^(m_w - M) and
+    // the weighted sum L, once (8 threads), for all D outputs of the head
+    if (tid < 8) {
+      float M = -kInf;
+#pragma unroll
+      for (int w = 0; w < NW; ++w) M = fmaxf(M, slots[w * S::WPART + tid]);
+      float L = 0.f;
+#pragma unroll
+      for (int w = 0; w < NW; ++w) {
+        const float e = M == -kInf ? 0.f : fast_exp2(slots[w * S::WPART + tid] - M);
+        s_wt[w][tid] = e;
+        L += e * slots[w * S::WPART + 8 + tid];
+      }
+      s_ml[0][tid] = M;
+      s_ml[1][tid] = L;
+    }
+    __syncthreads();
     const bool alone = c_first == c_last;
     float* gpart = p.ws_part + (static_cast<size_t>(u) + c) * S::WPART;
     for (int idx = tid; idx < 8 * D; idx += NT) {
       const int hh = idx / D, d = idx - hh * D;
-      float M = -kInf;
+      const float M = s_ml[0][hh], L = s_ml[1][hh];
+      float acc = 0.f;
 #pragma unroll
-      for (int w = 0; w < NW; ++w) M = fmaxf(M, slots[w * S::WPART + hh]);
-      float L = 0.f, acc = 0.f;
-      if (M != -kInf) {
-#pragma unroll
-        for (int w = 0; w < NW; ++w) {
-          const float e = fast_exp2(slots[w * S::WPART + hh] - M);
-          L += e * slots[w * S::WPART + 8 + hh];
-          acc += e * slots[w * S::WPART + 16 + hh * D + d];
-        }
-      }
+      for (int w = 0; w < NW; ++w) acc += s_wt[w][hh] * slots[w * S::WPART + 16 + hh * D + d];
       if (alone) {
         const int qi = grp * 8 + hh;
         if (qi < p.G) {
