@@ -188,15 +188,62 @@ kvq_status make_maps(int fmt, const kvq_cache* c, void* buf, CUtensorMap* tile, 
   return s;
 }
 
+// The four tensor maps of a cache (K tile, V tile, K scales, V scales), from
+// a small per-thread cache keyed by everything they encode: a decode step
+// reuses the maps of the previous step instead of re-encoding them.
+struct MapEntry {
+  int32_t fmt, H, D;
+  int64_t nb;
+  const void* k;
+  const void* v;
+  int dev;
+  CUtensorMap maps[4];
+};
+kvq_status cached_maps(int fmt, const kvq_cache* c, const CUtensorMap** out) {
+  constexpr int kEntries = 8;
+  thread_local MapEntry entries[kEntries];
+  thread_local int n_used = 0, next = 0;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) dev = -1;
+  for (int i = 0; i < n_used; ++i) {
+    const MapEntry& e = entries[i];
+    if (e.fmt == fmt && e.H == c->num_kv_heads && e.D == c->head_dim && e.nb == c->num_blocks &&
+        e.k == c->k && e.v == c->v && e.dev == dev) {
+      *out = e.maps;
+      return KVQ_OK;
+    }
+  }
+  MapEntry& e = entries[next];
+  e.k = nullptr;  // invalid until both encodes succeed
+  kvq_status s = make_maps(fmt, c, c->k, &e.maps[0], &e.maps[2]);
+  if (s != KVQ_OK) return s;
+  s = make_maps(fmt, c, c->v, &e.maps[1], &e.maps[3]);
+  if (s != KVQ_OK) return s;
+  e.fmt = fmt;
+  e.H = c->num_kv_heads;
+  e.D = c->head_dim;
+  e.nb = c->num_blocks;
+  e.k = c->k;
+  e.v = c->v;
+  e.dev = dev;
+  *out = e.maps;
+  if (n_used < kEntries) ++n_used;
+  next = (next + 1) % kEntries;
+  return KVQ_OK;
+}
+
 }  // namespace
 
 namespace kvq {
 void set_last_error(const char* msg) { snprintf(g_err, sizeof(g_err), "%s", msg); }
 
 int num_sms() {
+  static std::atomic<int> cached[64];  // per device ordinal; 0 = not yet asked
   int dev = 0, n = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (dev >= 0 && dev < 64 && (n = cached[dev].load(std::memory_order_relaxed)) > 0) return n;
   if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 148;
+  if (dev >= 0 && dev < 64) cached[dev].store(n, std::memory_order_relaxed);
   return n;
 }
 }  // namespace kvq
@@ -354,10 +401,8 @@ kvq_status kv_decode_attention(int32_t fmt, const void* q, const kvq_cache* cach
       return fail(KVQ_ERR_WORKSPACE, "workspace %zu bytes < %zu needed", workspace_bytes,
                   pl.ws_bytes);
   }
-  CUtensorMap maps[4];
-  s = make_maps(fmt, cache, cache->k, &maps[0], &maps[2]);
-  if (s != KVQ_OK) return s;
-  s = make_maps(fmt, cache, cache->v, &maps[1], &maps[3]);
+  const CUtensorMap* maps = nullptr;
+  s = cached_maps(fmt, cache, &maps);
   if (s != KVQ_OK) return s;
 
   kvq::DecodeParams p;
