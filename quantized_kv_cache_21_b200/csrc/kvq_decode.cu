@@ -56,7 +56,6 @@ constexpr float kLog2e = 1.4426950408889634f;
 // same factor.  A warp's running max m lags the true max by at most
 // kRescaleGap (log2 units): p <= 2^3, P <= 2^15 < 65504, the largest f16.
 constexpr float kPLog2 = 12.0f;
-constexpr float kPScale = 4096.0f;  // 2^kPLog2
 constexpr float kRescaleGap = 3.0f;
 constexpr float kETop = kPLog2 + kRescaleGap;  // e = s - m + kPLog2 above this moves m
 
