@@ -86,6 +86,9 @@ def lib():
         L.orc_decode_attention.restype = i32
         L.orc_decode_attention.argtypes = [i32, P, P, P, i64, i32, i32, P, i32, P, i32, i32,
                                            f32, f32, f64, P, i64, P, P]
+        L.orc_decode_attention_window.restype = i32
+        L.orc_decode_attention_window.argtypes = [i32, P, P, P, i64, i32, i32, P, i32, P, i32,
+                                                  i32, f32, f32, f64, i32, P, i64, P, P]
         L.orc_merge.restype = None
         L.orc_merge.argtypes = [i32, i32, P, P, P, P, P]
         _lib = L
@@ -201,11 +204,13 @@ def dequantize(fmt: str, k_cache, v_cache, H: int, D: int, slots, k_scale, v_sca
 
 
 def decode_attention(fmt: str, q_bits, k_cache, v_cache, H: int, block_table, seq_lens,
-                     k_scale, v_scale, sm_scale=None, pairs=None):
+                     k_scale, v_scale, sm_scale=None, pairs=None, window=0):
     """Float64 decode attention.  q_bits: [B][Hq][D] BF16 bit patterns;
     block_table [B][max_blocks] int32; seq_lens [B] int32.  Returns
     (out [B][Hq][D], lse [B][Hq]) in float64.  With ``pairs`` (an [n][2] array
-    of (b, j)), only those rows are computed and the rest are NaN."""
+    of (b, j)), only those rows are computed and the rest are NaN.  With
+    ``window`` > 0, sequence b attends only to its last ``window`` tokens (the
+    sliding-window mode of the MI300X benchmark page, section "SWA mode")."""
     q = _c(q_bits, np.uint16)
     B, Hq, D = q.shape
     bt = _c(block_table, np.int32)
@@ -220,10 +225,10 @@ def decode_attention(fmt: str, q_bits, k_cache, v_cache, H: int, block_table, se
     else:
         pr = _c(pairs, np.int32).reshape(-1, 2)
         pp, npairs = _p(pr), pr.shape[0]
-    rc = lib().orc_decode_attention(FORMATS[fmt], _p(q), _p(k_cache), _p(v_cache), nb, H, D,
-                                    _p(bt), bt.shape[1], _p(sl), B, Hq, float(k_scale),
-                                    float(v_scale), float(sm_scale), pp, npairs, _p(out),
-                                    _p(lse))
+    rc = lib().orc_decode_attention_window(FORMATS[fmt], _p(q), _p(k_cache), _p(v_cache), nb,
+                                           H, D, _p(bt), bt.shape[1], _p(sl), B, Hq,
+                                           float(k_scale), float(v_scale), float(sm_scale),
+                                           int(window), pp, npairs, _p(out), _p(lse))
     if rc:
         raise ValueError(f"oracle attention failed ({rc})")
     return out, lse

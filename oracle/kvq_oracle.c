@@ -414,6 +414,42 @@ int orc_attention_range(int fmt, const uint16_t* q_row, const void* k_cache, con
 }
 
 /*
+ * Decode step over a sliding window ("AMD MI300X — KV Cache Compression
+ * Benchmark", section "SWA mode": only the most recent `window` tokens of the
+ * cache are attended to).  Sequence b attends to its tokens
+ * [max(0, len_b - window), len_b); window <= 0 means the whole context.
+ * Otherwise as orc_decode_attention below.
+ */
+int orc_decode_attention_window(int fmt, const uint16_t* q, const void* k_cache,
+                                const void* v_cache, int64_t num_blocks, int H, int D,
+                                const int32_t* block_table, int max_blocks,
+                                const int32_t* seq_lens, int B, int Hq, float k_scale,
+                                float v_scale, double sm_scale, int32_t window,
+                                const int32_t* pairs, int64_t n_pairs, double* out, double* lse) {
+  int G = Hq / H;
+  int64_t total = pairs ? n_pairs : (int64_t)B * Hq;
+  for (int64_t i = 0; i < total; i++) {
+    int b = pairs ? pairs[2 * i] : (int)(i / Hq);
+    int j = pairs ? pairs[2 * i + 1] : (int)(i % Hq);
+    int64_t len = seq_lens[b];
+    int64_t t0 = (window > 0 && len > window) ? len - window : 0;
+    double m, l;
+    double* o = out + ((int64_t)b * Hq + j) * D;
+    int rc = orc_attention_range(fmt, q + ((int64_t)b * Hq + j) * D, k_cache, v_cache, num_blocks,
+                                 H, D, block_table + (int64_t)b * max_blocks, j / G, t0, len,
+                                 k_scale, v_scale, sm_scale, o, &m, &l);
+    if (rc) return rc;
+    if (l > 0.0) {
+      for (int d = 0; d < D; d++) o[d] /= l;
+      lse[(int64_t)b * Hq + j] = m + log(l);
+    } else {
+      lse[(int64_t)b * Hq + j] = -INFINITY;
+    }
+  }
+  return 0;
+}
+
+/*
  * Full decode step: out[b][j][:] = o_unnorm / l and lse[b][j] = m + ln(l) for
  * every sequence b and query head j (natural log, scaled-score units).  A
  * sequence of length 0 gives out = 0 and lse = -inf.  q is [B][Hq][D] BF16;
@@ -426,25 +462,9 @@ int orc_decode_attention(int fmt, const uint16_t* q, const void* k_cache, const 
                          int max_blocks, const int32_t* seq_lens, int B, int Hq, float k_scale,
                          float v_scale, double sm_scale, const int32_t* pairs, int64_t n_pairs,
                          double* out, double* lse) {
-  int G = Hq / H;
-  int64_t total = pairs ? n_pairs : (int64_t)B * Hq;
-  for (int64_t i = 0; i < total; i++) {
-    int b = pairs ? pairs[2 * i] : (int)(i / Hq);
-    int j = pairs ? pairs[2 * i + 1] : (int)(i % Hq);
-    double m, l;
-    double* o = out + ((int64_t)b * Hq + j) * D;
-    int rc = orc_attention_range(fmt, q + ((int64_t)b * Hq + j) * D, k_cache, v_cache, num_blocks,
-                                 H, D, block_table + (int64_t)b * max_blocks, j / G, 0,
-                                 seq_lens[b], k_scale, v_scale, sm_scale, o, &m, &l);
-    if (rc) return rc;
-    if (l > 0.0) {
-      for (int d = 0; d < D; d++) o[d] /= l;
-      lse[(int64_t)b * Hq + j] = m + log(l);
-    } else {
-      lse[(int64_t)b * Hq + j] = -INFINITY;
-    }
-  }
-  return 0;
+  return orc_decode_attention_window(fmt, q, k_cache, v_cache, num_blocks, H, D, block_table,
+                                     max_blocks, seq_lens, B, Hq, k_scale, v_scale, sm_scale, 0,
+                                     pairs, n_pairs, out, lse);
 }
 
 /*

@@ -142,3 +142,74 @@ def test_page_placement_invariance():
     ob = oracle.decode_attention("nvfp4", b["q"], b["kc"], b["vc"], H, b["bt"], b["lens"],
                                  b["ks"], b["vs"])
     assert np.array_equal(oa[0], ob[0]) and np.array_equal(oa[1], ob[1])
+
+
+# ---- sliding-window mode ("AMD MI300X — KV Cache Compression Benchmark",
+# section "SWA mode": attention over the most recent `window` tokens)
+
+@pytest.mark.parametrize("fmt", ["bf16", "fp8", "nvfp4"])
+def test_window_matches_torch_sdpa_on_the_last_tokens(fmt):
+    """torch float64 SDPA over only the last W dequantised tokens (W < len,
+    W = len, W > len, and a W that is not a multiple of the page size)."""
+    B, H, Hq, D = 4, 2, 8, 64
+    c = build_case(fmt, B, H, Hq, D, [100, 37, 16, 70], seed=700, factor=8.0)
+    G = Hq // H
+    for W in (1, 17, 37, 64, 500):
+        out, lse = oracle.decode_attention(fmt, c["q"], c["kc"], c["vc"], H, c["bt"], c["lens"],
+                                           c["ks"], c["vs"], window=W)
+        for b in range(B):
+            n = int(c["lens"][b])
+            t0 = max(0, n - W)
+            kd, vd = dequant_seq(fmt, c, b)
+            k = torch.from_numpy(kd[t0:].astype(np.float64)).permute(1, 0, 2).repeat_interleave(G, 0)
+            v = torch.from_numpy(vd[t0:].astype(np.float64)).permute(1, 0, 2).repeat_interleave(G, 0)
+            q = torch.from_numpy(wl.bf16_bits_to_f32(c["q"][b]).astype(np.float64))[:, None, :]
+            ref = torch.nn.functional.scaled_dot_product_attention(q, k, v)[:, 0, :]
+            scores = (q @ k.transpose(1, 2))[:, 0, :] / math.sqrt(D)
+            np.testing.assert_allclose(out[b], ref.numpy(), rtol=1e-12, atol=1e-12)
+            np.testing.assert_allclose(lse[b], torch.logsumexp(scores, -1).numpy(), rtol=1e-12)
+
+
+def test_window_equals_full_attention_over_a_truncated_cache():
+    """A windowed decode over the cache equals a full decode over a cache that
+    holds only those last W tokens (the page's truncated-cache form), with the
+    tokens at other pages and offsets."""
+    fmt, B, H, Hq, D, W = "fp8", 2, 2, 8, 128, 45
+    c = build_case(fmt, B, H, Hq, D, [200, 30], seed=701, factor=4.0)
+    out_w, lse_w = oracle.decode_attention(fmt, c["q"], c["kc"], c["vc"], H, c["bt"], c["lens"],
+                                           c["ks"], c["vs"], window=W)
+    rng = wl.rng_for(702, 0)
+    for b in range(B):
+        n = int(c["lens"][b])
+        t0 = max(0, n - W)
+        # the raw codes of the last W tokens, rewritten at positions 0.. of a
+        # fresh randomly permuted table (codes are copied, not re-quantized)
+        m = n - t0
+        nbps = -(-m // 16)
+        bt2 = wl.permuted_block_table(rng, 1, nbps, nbps + 5)
+        kc2, vc2 = oracle.new_cache(fmt, nbps + 5, H, D)
+        page = oracle.head_page_bytes(fmt, D)
+        src = wl.physical_slots(c["bt"], b, np.arange(t0, n))
+        dst = wl.physical_slots(bt2, 0, np.arange(m))
+        for s_, d_ in zip(src, dst):
+            for h in range(H):
+                so = (s_ // 16 * H + h) * page + (s_ % 16) * D
+                do = (d_ // 16 * H + h) * page + (d_ % 16) * D
+                kc2[do:do + D] = c["kc"][so:so + D]
+                vc2[do:do + D] = c["vc"][so:so + D]
+        out_f, lse_f = oracle.decode_attention(fmt, c["q"][b:b + 1], kc2, vc2, H, bt2,
+                                               np.array([m], np.int32), c["ks"], c["vs"])
+        assert np.array_equal(out_w[b], out_f[0]) and np.array_equal(lse_w[b], lse_f[0])
+
+
+def test_window_of_one_token_returns_the_last_value():
+    fmt, H, Hq, D = "bf16", 1, 4, 64
+    c = build_case(fmt, 1, H, Hq, D, [50], seed=703)
+    out, lse = oracle.decode_attention(fmt, c["q"], c["kc"], c["vc"], H, c["bt"], c["lens"],
+                                       c["ks"], c["vs"], window=1)
+    kd, vd = dequant_seq(fmt, c, 0)
+    q = wl.bf16_bits_to_f32(c["q"][0]).astype(np.float64)
+    for j in range(Hq):
+        np.testing.assert_array_equal(out[0, j], vd[-1, 0].astype(np.float64))
+        assert lse[0, j] == pytest.approx(q[j] @ kd[-1, 0].astype(np.float64) / math.sqrt(D),
+                                          rel=1e-12)
