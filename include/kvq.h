@@ -209,6 +209,31 @@ kvq_status kv_decode_attention(int32_t fmt, const void* q, const kvq_cache* cach
                                void* workspace, size_t workspace_bytes, int32_t* d_err,
                                kvq_stream stream);
 
+/* kv_decode_attention in sliding-window mode ("AMD MI300X — KV Cache
+ * Compression Benchmark", section "SWA mode": attention over the most recent
+ * `window` tokens of a truncated or windowed cache).  Sequence b attends to
+ * its tokens [max(0, seq_lens[b] - window), seq_lens[b]) only; window = 0 is
+ * kv_decode_attention itself.  The work is split over the window's pages
+ * only, so a short window over a long cache reads ~window tokens per
+ * sequence.  Same arguments, layouts and errors as kv_decode_attention;
+ * window < 0 is KVQ_ERR_INVALID_ARG.  The workspace must hold
+ * kv_decode_workspace_size_window() bytes for the same arguments. */
+kvq_status kv_decode_attention_window(int32_t fmt, const void* q, const kvq_cache* cache,
+                                      const int32_t* block_table, int32_t max_blocks,
+                                      const int32_t* seq_lens, int32_t num_seqs,
+                                      int32_t num_q_heads, int32_t max_seq_len, int32_t window,
+                                      int32_t num_splits, const float* d_k_scale,
+                                      const float* d_v_scale, float sm_scale, float* out,
+                                      float* lse, void* workspace, size_t workspace_bytes,
+                                      int32_t* d_err, kvq_stream stream);
+
+/* Workspace bytes kv_decode_attention_window needs (as
+ * kv_decode_workspace_size, with the window). */
+kvq_status kv_decode_workspace_size_window(int32_t fmt, int32_t num_seqs, int32_t num_q_heads,
+                                           int32_t num_kv_heads, int32_t head_dim,
+                                           int32_t max_seq_len, int32_t window,
+                                           int32_t num_splits, size_t* bytes);
+
 /* kv_decode_attention without a caller workspace, for callers that cannot
  * allocate device memory when they run a decode step (their device memory
  * belongs to a fixed pool they must not bypass, they may not pay a

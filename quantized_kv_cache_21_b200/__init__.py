@@ -32,7 +32,7 @@ DERR_TIMEOUT = 0x10
 EXPORTS = ("kvq_status_string", "kvq_last_error", "kv_cache_bytes", "kv_scale_from_absmax",
            "kv_scale_from_absmax_device", "kv_calibrate_absmax", "kv_quantize_write",
            "kv_decode_workspace_size", "kv_decode_attention", "kv_decode_attention_static_ws",
-           "kv_dequantize")
+           "kv_decode_attention_window", "kv_decode_workspace_size_window", "kv_dequantize")
 
 
 class KvqError(RuntimeError):
@@ -73,6 +73,10 @@ def lib() -> ctypes.CDLL:
                                     P, sz, P, P],
             "kv_decode_attention_static_ws": [i32, P, CP, P, i32, P, i32, i32, i32, i32, P, P,
                                               f32, P, P, P, P],
+            "kv_decode_attention_window": [i32, P, CP, P, i32, P, i32, i32, i32, i32, i32, P, P,
+                                           f32, P, P, P, sz, P, P],
+            "kv_decode_workspace_size_window": [i32, i32, i32, i32, i32, i32, i32, i32,
+                                                ctypes.POINTER(sz)],
             "kv_dequantize": [i32, CP, P, i64, P, P, P, P, P, P],
         }
         for name, args in sigs.items():
@@ -221,6 +225,36 @@ def kv_decode_attention_static_ws(fmt, q: torch.Tensor, cache: KVCache,
                                                max_seq_len, num_splits, _ptr(k_scale),
                                                _ptr(v_scale), float(sm_scale), _ptr(out),
                                                _ptr(lse), _ptr(d_err), _stream(stream)))
+
+
+def kv_decode_workspace_size_window(fmt, num_seqs: int, num_q_heads: int, num_kv_heads: int,
+                                    head_dim: int, max_seq_len: int, window: int,
+                                    num_splits: int = 0) -> int:
+    out = ctypes.c_size_t()
+    _check(lib().kv_decode_workspace_size_window(_fmt(fmt), num_seqs, num_q_heads, num_kv_heads,
+                                                 head_dim, max_seq_len, window, num_splits,
+                                                 ctypes.byref(out)))
+    return out.value
+
+
+def kv_decode_attention_window(fmt, q: torch.Tensor, cache: KVCache, block_table: torch.Tensor,
+                               seq_lens: torch.Tensor, max_seq_len: int, window: int, k_scale,
+                               v_scale, out: torch.Tensor, lse: torch.Tensor | None,
+                               workspace: torch.Tensor | None, d_err: torch.Tensor | None = None,
+                               sm_scale: float = 0.0, num_splits: int = 0, stream=None):
+    """kv_decode_attention over each sequence's last ``window`` tokens only
+    (sliding-window mode; see include/kvq.h)."""
+    assert q.dtype == torch.bfloat16 and q.is_contiguous()
+    assert block_table.dtype == torch.int32 and seq_lens.dtype == torch.int32
+    assert out.dtype == torch.float32
+    B, Hq, _ = q.shape
+    ws_bytes = workspace.numel() if workspace is not None else 0
+    _check(lib().kv_decode_attention_window(_fmt(fmt), _ptr(q), cache.c, _ptr(block_table),
+                                            block_table.shape[1], _ptr(seq_lens), B, Hq,
+                                            max_seq_len, window, num_splits, _ptr(k_scale),
+                                            _ptr(v_scale), float(sm_scale), _ptr(out), _ptr(lse),
+                                            _ptr(workspace), ws_bytes, _ptr(d_err),
+                                            _stream(stream)))
 
 
 def kv_dequantize(fmt, cache: KVCache, slots: torch.Tensor, k_scale, v_scale,

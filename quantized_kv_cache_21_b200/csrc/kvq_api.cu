@@ -85,7 +85,7 @@ struct Plan {
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 kvq_status make_plan(int32_t fmt, int32_t B, int32_t Hq, int32_t Hkv, int32_t D,
-                     int32_t max_seq_len, int32_t num_splits, Plan* pl) {
+                     int32_t max_seq_len, int32_t num_splits, Plan* pl, int32_t window = 0) {
   kvq::DecodeConfig cfg;
   if (fmt < 0 || fmt > 2 || !kvq::decode_config(fmt, D, &cfg))
     return fail(KVQ_ERR_UNSUPPORTED, "format %d / head_dim %d", fmt, D);
@@ -99,6 +99,11 @@ kvq_status make_plan(int32_t fmt, int32_t B, int32_t Hq, int32_t Hkv, int32_t D,
   if (units > 0x7fffffff) return fail(KVQ_ERR_UNSUPPORTED, "too many (sequence, head) units");
   pl->units = (int)units;
   pl->pmax = (max_seq_len + KVQ_BLOCK_SIZE - 1) / KVQ_BLOCK_SIZE;
+  if (window < 0) return fail(KVQ_ERR_INVALID_ARG, "window %d", window);
+  if (window > 0) {  // a window's tokens span at most ceil(window / 16) + 1 pages
+    const int wp = (window + KVQ_BLOCK_SIZE - 1) / KVQ_BLOCK_SIZE + 1;
+    if (wp < pl->pmax) pl->pmax = wp;
+  }
   const int64_t V = units * pl->pmax;
   const int sms = kvq::num_sms();
   int64_t ctas;
@@ -365,6 +370,21 @@ kvq_status kv_decode_workspace_size(int32_t fmt, int32_t num_seqs, int32_t num_q
   return KVQ_OK;
 }
 
+kvq_status kv_decode_workspace_size_window(int32_t fmt, int32_t num_seqs, int32_t num_q_heads,
+                                           int32_t num_kv_heads, int32_t head_dim,
+                                           int32_t max_seq_len, int32_t window,
+                                           int32_t num_splits, size_t* bytes) {
+  if (!bytes) return fail(KVQ_ERR_INVALID_ARG, "bytes is NULL");
+  kvq_status s = check_device();
+  if (s != KVQ_OK) return s;
+  Plan pl;
+  s = make_plan(fmt, num_seqs, num_q_heads, num_kv_heads, head_dim, max_seq_len, num_splits, &pl,
+                window);
+  if (s != KVQ_OK) return s;
+  *bytes = pl.ws_bytes;
+  return KVQ_OK;
+}
+
 kvq_status kv_decode_attention(int32_t fmt, const void* q, const kvq_cache* cache,
                                const int32_t* block_table, int32_t max_blocks,
                                const int32_t* seq_lens, int32_t num_seqs, int32_t num_q_heads,
@@ -372,6 +392,19 @@ kvq_status kv_decode_attention(int32_t fmt, const void* q, const kvq_cache* cach
                                const float* d_v_scale, float sm_scale, float* out, float* lse,
                                void* workspace, size_t workspace_bytes, int32_t* d_err,
                                kvq_stream stream) {
+  return kv_decode_attention_window(fmt, q, cache, block_table, max_blocks, seq_lens, num_seqs,
+                                    num_q_heads, max_seq_len, 0, num_splits, d_k_scale, d_v_scale,
+                                    sm_scale, out, lse, workspace, workspace_bytes, d_err, stream);
+}
+
+kvq_status kv_decode_attention_window(int32_t fmt, const void* q, const kvq_cache* cache,
+                                      const int32_t* block_table, int32_t max_blocks,
+                                      const int32_t* seq_lens, int32_t num_seqs,
+                                      int32_t num_q_heads, int32_t max_seq_len, int32_t window,
+                                      int32_t num_splits, const float* d_k_scale,
+                                      const float* d_v_scale, float sm_scale, float* out,
+                                      float* lse, void* workspace, size_t workspace_bytes,
+                                      int32_t* d_err, kvq_stream stream) {
   kvq_status s = check_cache(fmt, cache);
   if (s != KVQ_OK) return s;
   const int D = cache->head_dim, Hkv = cache->num_kv_heads;
@@ -391,7 +424,7 @@ kvq_status kv_decode_attention(int32_t fmt, const void* q, const kvq_cache* cach
   s = check_device();
   if (s != KVQ_OK) return s;
   Plan pl;
-  s = make_plan(fmt, num_seqs, num_q_heads, Hkv, D, max_seq_len, num_splits, &pl);
+  s = make_plan(fmt, num_seqs, num_q_heads, Hkv, D, max_seq_len, num_splits, &pl, window);
   if (s != KVQ_OK) return s;
   if (pl.ws_bytes > 0) {
     if (!workspace || !aligned(workspace, 256))
@@ -427,6 +460,7 @@ kvq_status kv_decode_attention(int32_t fmt, const void* q, const kvq_cache* cach
   p.units = pl.units;
   p.pmax = pl.pmax;
   p.max_seq_len = max_seq_len;
+  p.window = window;
   p.sm_scale = sm_scale;
   cudaError_t e = kvq::launch_decode(fmt, D, maps, p, pl.ctas, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? KVQ_OK : cuda_fail(e, "decode kernel");

@@ -563,8 +563,16 @@ __device__ __forceinline__ int cta_of(int64_t g, int64_t V, int C) {
 
 struct UnitView {
   int b, h, grp, len;
-  int ps, pe;  // this CTA's page range of the unit, clipped to its length
+  int first;   // absolute page of the attended range's first token (window mode)
+  int ps, pe;  // this CTA's page range of the unit (relative to first), clipped
 };
+
+// First page of the attended tokens of a sequence of length len: with a
+// sliding window, the tokens [len - window, len) ("AMD MI300X — KV Cache
+// Compression Benchmark", section "SWA mode"); else page 0.
+__device__ __forceinline__ int window_first(const DecodeParams& p, int len) {
+  return (p.window > 0 && len > p.window) ? (len - p.window) / kPage : 0;
+}
 
 __device__ __forceinline__ int ps_of(const DecodeParams& p, int u, int64_t vbeg) {
   const int64_t base = static_cast<int64_t>(u) * p.pmax;
@@ -580,8 +588,9 @@ __device__ __forceinline__ UnitView unit_view(const DecodeParams& p, int u, int6
   int len = __ldg(p.seq_lens + v.b);
   if (len < 0 || len > p.max_seq_len) len = 0;  // reported by the unit's first CTA
   v.len = len;
+  v.first = window_first(p, len);
   const int64_t base = static_cast<int64_t>(u) * p.pmax;
-  const int npages = (len + kPage - 1) / kPage;
+  const int npages = (len + kPage - 1) / kPage - v.first;
   v.ps = ps_of(p, u, vbeg);
   const int pe = static_cast<int>((vend < base + p.pmax ? vend : base + p.pmax) - base);
   v.pe = pe < npages ? pe : npages;
@@ -596,6 +605,7 @@ struct UnitTable {
   int n, total;
   int kend[kMaxUnits];
   int len[kMaxUnits];
+  int first[kMaxUnits];
 };
 
 // Block id and KV head of the CTA's item k, or blk = -1 past the last item.
@@ -604,7 +614,7 @@ __device__ __forceinline__ void item_block(const DecodeParams& p, const UnitTabl
   blk = -1;
   h = 0;
   if (k >= tab.total) return;
-  int i = 0, k0 = 0;
+  int i = 0, k0 = 0, first = 0;
   if (tab.n <= kMaxUnits) {
     int lo = 0, hi = tab.n - 1;
     while (lo < hi) {
@@ -616,9 +626,11 @@ __device__ __forceinline__ void item_block(const DecodeParams& p, const UnitTabl
     }
     i = lo;
     k0 = i ? tab.kend[i - 1] : 0;
+    first = tab.first[i];
   } else {  // long unit lists: walk them
     for (;;) {
       const UnitView uv = unit_view(p, u0 + i, vbeg, vend);
+      first = uv.first;
       if (k < k0 + uv.pe - uv.ps) break;
       k0 += uv.pe - uv.ps;
       ++i;
@@ -627,7 +639,8 @@ __device__ __forceinline__ void item_block(const DecodeParams& p, const UnitTabl
   const int u = u0 + i;
   h = (u / p.n_groups) % p.Hkv;
   const int b = u / (p.n_groups * p.Hkv);
-  blk = __ldg(p.block_table + static_cast<size_t>(b) * p.max_blocks + ps_of(p, u, vbeg) + (k - k0));
+  blk = __ldg(p.block_table + static_cast<size_t>(b) * p.max_blocks + first + ps_of(p, u, vbeg) +
+              (k - k0));
 }
 
 // Merge the per-CTA partials of unit u (slots u + c for c in [c_first,
@@ -792,11 +805,12 @@ __global__ void __launch_bounds__(Shape<FMT, D>::NW * 32, 1)
     int run = 0;
     for (int base = 0; base < nu; base += 32) {
       const int i = base + lane;
-      int n_i = 0, len_i = 0;
+      int n_i = 0, len_i = 0, first_i = 0;
       if (i < nu) {
         const UnitView uv = unit_view(p, u0 + i, vbeg, vend);
         n_i = scale_ok ? uv.pe - uv.ps : 0;
         len_i = uv.len;
+        first_i = uv.first;
       }
       int x = n_i;
 #pragma unroll
@@ -807,6 +821,7 @@ __global__ void __launch_bounds__(Shape<FMT, D>::NW * 32, 1)
       if (i < nu && i < kMaxUnits) {
         tab.kend[i] = run + x;
         tab.len[i] = len_i;
+        tab.first[i] = first_i;
       }
       run += __shfl_sync(0xffffffffu, x, 31);
     }
@@ -817,7 +832,7 @@ __global__ void __launch_bounds__(Shape<FMT, D>::NW * 32, 1)
   }
   // Ask L2 for the pages of this warp's first stages (the guessed block ids)
   // while the unit table is built; a wrong guess only costs a prefetch.
-  if (lane < NSW && spec0 >= 0 && spec0 < p.num_blocks)
+  if (p.window <= 0 && lane < NSW && spec0 >= 0 && spec0 < p.num_blocks)
     F::prefetch(&mk, &mv, (u0 / p.n_groups) % p.Hkv, spec0);
   if (lane < NSW) mbar_init(&bars[lane], 1);  // each warp its own stages
   mbar_init_fence();
@@ -834,7 +849,8 @@ __global__ void __launch_bounds__(Shape<FMT, D>::NW * 32, 1)
   int chunk = 0;
   int cur_blk, cur_h, nxt_blk, nxt_h;
   {
-    const int k_first = tab.kend[0], h0 = (u0 / p.n_groups) % p.Hkv;
+    // the guess assumes the unit's pages start at page 0 (no window)
+    const int k_first = p.window > 0 ? 0 : tab.kend[0], h0 = (u0 / p.n_groups) % p.Hkv;
     if (g0 < k_first) {
       cur_blk = spec0;
       cur_h = h0;
@@ -901,14 +917,16 @@ __global__ void __launch_bounds__(Shape<FMT, D>::NW * 32, 1)
   for (int si = 0; si < nu; ++si) {
     const int u = u0 + si;
     const int grp = u % p.n_groups, h = (u / p.n_groups) % p.Hkv, b = u / (p.n_groups * p.Hkv);
-    int n_items, len;
+    int n_items, len, first;
     if (nu <= kMaxUnits) {
       n_items = tab.kend[si] - (si ? tab.kend[si - 1] : 0);
       len = tab.len[si];
+      first = tab.first[si];
     } else {
       const UnitView uv = unit_view(p, u, vbeg, vend);
       n_items = scale_ok ? uv.pe - uv.ps : 0;
       len = uv.len;
+      first = uv.first;
     }
     const int ps = ps_of(p, u, vbeg);
     const int c_first = cta_of(static_cast<int64_t>(u) * p.pmax, V, C);
@@ -927,7 +945,10 @@ __global__ void __launch_bounds__(Shape<FMT, D>::NW * 32, 1)
 
     const int k_end = k_base + n_items;
     // valid tokens of the segment's last page (only that page can be partial)
-    const int n_last = len - (ps + n_items - 1) * kPage;
+    const int n_last = len - (first + ps + n_items - 1) * kPage;
+    // window mode: tokens of the window's first page before its start are
+    // masked (only the unit's relative page 0 can hold such tokens)
+    const int n_skip = (p.window > 0 && len > p.window) ? len - p.window - first * kPage : 0;
     for (int k = warp + j * NW; k < k_end; k += NW, ++j) {
       const uint8_t* sp = ring + st * F::STAGE;
       // all lanes agree on the outcome so the warp stays converged
@@ -993,6 +1014,10 @@ __global__ void __launch_bounds__(Shape<FMT, D>::NW * 32, 1)
           va[jj][2] &= m23;
           va[jj][3] &= m23;
         }
+      }
+      if (n_skip > 0 && ps == 0 && k == k_base) {  // window's first page: tokens before it
+        if (gid < n_skip) r0 = r1 = -kInf;
+        if (gid + 8 < n_skip) r2 = r3 = -kInf;
       }
 
       // ---- online softmax (log2 domain); this thread: heads 2tig, 2tig+1.

@@ -26,6 +26,7 @@ struct DecodeParams {
   int units;                  // B * Hkv * n_groups (sequence, KV head, group of 8 q heads)
   int pmax;                   // pages per unit in the work partition: ceil(max_seq_len / 16)
   int max_seq_len;
+  int window;                 // > 0: attend to each sequence's last `window` tokens only
   float sm_scale;
 };
 
