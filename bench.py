@@ -519,6 +519,23 @@ def main():
                                  for f in ("fp8", "nvfp4")}
         line["agents_formats"] = af
 
+        # sliding-window mode ("SWA mode" of the MI300X benchmark page: window
+        # 4096) on the main workload's cache: decode launches only
+        s5 = DecodeScenario(w, device="cuda")
+        swa = {}
+        for win in (4096,):
+            s5.window_ws(win)
+            (dms,), _ = timer.run([lambda: s5.decode_window(win)], K, W)
+            b5 = s5.window_scan_bytes(win)
+            a = b5 / (statistics.mean(dms) * 1e-3) / 1e9
+            swa[str(win)] = {"us_per_step": statistics.mean(dms) * 1e3, "kv_scan_bytes": b5,
+                             "GBps": a, "frac_of_hbm_peak": a / peak}
+        assert int(s5.err.item()) == 0
+        line["sliding_window"] = {"config": dict(workload_config(w), window="last 4096 tokens"),
+                                  "windows": swa}
+        del s5
+        torch.cuda.empty_cache()
+
         x = wl.device_tokens(20264, 0, 65536, 8, 128)
         amax = torch.zeros(1, dtype=torch.float32, device="cuda")
         (cms,), _ = timer.run([lambda: kvq.kv_calibrate_absmax(x, amax)], K, W)

@@ -123,6 +123,26 @@ class DecodeScenario:
                                 self.lse if lse is None else lse, self.ws, self.err,
                                 stream=stream)
 
+    def decode_window(self, window: int, stream=None, out=None, lse=None):
+        """Sliding-window decode over each sequence's last ``window`` tokens
+        (needs a workspace sized for the window: window_workspace())."""
+        kvq.kv_decode_attention_window(self.fmt, self.q, self.cache, self.d_bt, self.d_lens,
+                                       self.L, window, self.d_ks, self.d_vs,
+                                       self.out if out is None else out,
+                                       self.lse if lse is None else lse,
+                                       self.window_ws(window), self.err, stream=stream)
+
+    def window_ws(self, window: int):
+        ws = getattr(self, "_wws", {})
+        if window not in ws:
+            ws[window] = kvq.new_workspace(kvq.kv_decode_workspace_size_window(
+                self.fmt, self.B, self.Hq, self.H, self.D, self.L, window), device=self.device)
+            self._wws = ws
+        return ws[window]
+
+    def window_scan_bytes(self, window: int) -> int:
+        return kv_scan_bytes(self.fmt, np.minimum(self.lens, window), self.H, self.D)
+
     def step(self, stream=None):
         self.write(stream)
         self.decode(stream)
