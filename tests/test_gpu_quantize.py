@@ -37,10 +37,12 @@ def write_both(fmt, k, v, slots, nb, ks, vs, fill=0):
     return okc, ovc, gk, gv, int(err.item()), cache
 
 
-@pytest.mark.parametrize("scale", [1.0, 0.125, 3.0517578125e-05])
+@pytest.mark.parametrize("scale", [1.0, 0.125, 3.0517578125e-05, 0.0234375, 1e-12, 0.7,
+                                   33333.0, oracle.scale_from_absmax("fp8", 7.3)])
 def test_fp8_every_bf16_input(scale):
     """All 65,280 finite BF16 values through x / s -> E4M3 (s = 1 makes it the
-    bare encoder; the other scales move every value across binades)."""
+    bare encoder; the other scales move every value across binades; scales
+    that are not powers of two make x / s a true division)."""
     bits = all_finite_bf16()
     H, D = 1, 64
     T = bits.size // D  # 65280 = 1020 * 64
@@ -70,6 +72,55 @@ def test_e2m1_every_rounding_case():
     k = blocks.reshape(nrow, 1, D)
     slots = np.arange(nrow, dtype=np.int64)
     okc, ovc, gk, gv, err, _ = write_both("nvfp4", k, k, slots, -(-nrow // 16), 0.125, 0.125)
+    assert err == 0
+    assert np.array_equal(gk, okc) and np.array_equal(gv, ovc)
+
+
+def test_e2m1_every_rounding_case_with_an_inexact_divisor():
+    """As above with g = 0.1 and a block maximum of BF16(0.825): the block
+    scale encodes to 1.375 and every element is divided by 1.375 * fp32(0.1),
+    which is not a power of two, so each E2M1 input is a rounded quotient."""
+    bits = all_finite_bf16()
+    x = wl.bf16_bits_to_f32(bits)
+    top = wl.f32_to_bf16_bits(np.array([0.825], np.float32))[0]
+    vals = bits[np.abs(x) <= wl.bf16_bits_to_f32(np.array([top]))[0]]
+    per_block = 15
+    nblk = -(-vals.size // per_block)
+    vals = np.concatenate([vals, np.zeros(nblk * per_block - vals.size, np.uint16)])
+    blocks = np.concatenate([vals.reshape(nblk, per_block), np.full((nblk, 1), top, np.uint16)], 1)
+    D = 128
+    nrow = -(-nblk // (D // 16))
+    blocks = np.concatenate([blocks, np.zeros((nrow * (D // 16) - nblk, 16), np.uint16)])
+    k = blocks.reshape(nrow, 1, D)
+    slots = np.arange(nrow, dtype=np.int64)
+    g = float(np.float32(0.1))
+    okc, ovc, gk, gv, err, _ = write_both("nvfp4", k, k, slots, -(-nrow // 16), g, g)
+    assert err == 0
+    assert np.array_equal(gk, okc) and np.array_equal(gv, ovc)
+
+
+def test_e2m1_rounding_with_a_subnormal_divisor():
+    """g = 2^-130 (a subnormal fp32 scale) and a block maximum of 6 g: the block
+    scale decodes to 1, every element is divided by the subnormal 2^-130, and
+    the BF16 subnormals up to 6 g give the quotients k / 8 for k = 0..48, which
+    hit every E2M1 tie exactly (1/(2^-130) is not a finite fp32 number, so a
+    reciprocal-based division would not do)."""
+    g = 2.0 ** -130
+    bits = all_finite_bf16()
+    x = wl.bf16_bits_to_f32(bits)
+    top = wl.f32_to_bf16_bits(np.array([6 * g], np.float32))[0]
+    vals = bits[np.abs(x) <= 6 * g]
+    assert vals.size == 2 * 49  # +-k * 2^-133 for k = 0..48 (both zeros)
+    per_block = 15
+    nblk = -(-vals.size // per_block)
+    vals = np.concatenate([vals, np.zeros(nblk * per_block - vals.size, np.uint16)])
+    blocks = np.concatenate([vals.reshape(nblk, per_block), np.full((nblk, 1), top, np.uint16)], 1)
+    D = 64
+    nrow = -(-nblk // (D // 16))
+    blocks = np.concatenate([blocks, np.zeros((nrow * (D // 16) - nblk, 16), np.uint16)])
+    k = blocks.reshape(nrow, 1, D)
+    slots = np.arange(nrow, dtype=np.int64)
+    okc, ovc, gk, gv, err, _ = write_both("nvfp4", k, k, slots, 1, g, g)
     assert err == 0
     assert np.array_equal(gk, okc) and np.array_equal(gv, ovc)
 
