@@ -90,6 +90,9 @@ def lib():
         L.orc_decode_attention_window.argtypes = [i32, P, P, P, i64, i32, i32, P, i32, P, i32,
                                                   i32, f32, f32, f64, i32, P, i64, P, P]
         L.orc_merge.restype = None
+        L.orc_prefill_attention.restype = i32
+        L.orc_prefill_attention.argtypes = [i32, P, P, P, i64, i32, i32, P, i32, P, i32, i32,
+                                            i32, f32, f32, f64, P, i64, P, P]
         L.orc_merge.argtypes = [i32, i32, P, P, P, P, P]
         _lib = L
     return _lib
@@ -231,6 +234,36 @@ def decode_attention(fmt: str, q_bits, k_cache, v_cache, H: int, block_table, se
                                            int(window), pp, npairs, _p(out), _p(lse))
     if rc:
         raise ValueError(f"oracle attention failed ({rc})")
+    return out, lse
+
+
+def prefill_attention(fmt: str, q_bits, k_cache, v_cache, H: int, block_table, seq_lens,
+                      k_scale, v_scale, sm_scale=None, rows=None):
+    """Float64 chunked-prefill attention.  q_bits: [B][Tq][Hq][D] BF16 bit
+    patterns, the Tq newest tokens of each sequence; seq_lens [B] counts them.
+    Query token i of sequence b (position seq_lens[b] - Tq + i) attends to the
+    cache tokens up to and including its own position.  Returns (out
+    [B][Tq][Hq][D], lse [B][Tq][Hq]) in float64; with ``rows`` (an [n][3]
+    array of (b, i, j)) only those rows are computed and the rest are NaN."""
+    q = _c(q_bits, np.uint16)
+    B, Tq, Hq, D = q.shape
+    bt = _c(block_table, np.int32)
+    sl = _c(seq_lens, np.int32)
+    nb = k_cache.size // (H * head_page_bytes(fmt, D))
+    if sm_scale is None:
+        sm_scale = 1.0 / np.sqrt(D)
+    out = np.full((B, Tq, Hq, D), np.nan)
+    lse = np.full((B, Tq, Hq), np.nan)
+    if rows is None:
+        rp, nr = None, 0
+    else:
+        rr = _c(rows, np.int32).reshape(-1, 3)
+        rp, nr = _p(rr), rr.shape[0]
+    rc = lib().orc_prefill_attention(FORMATS[fmt], _p(q), _p(k_cache), _p(v_cache), nb, H, D,
+                                     _p(bt), bt.shape[1], _p(sl), B, Tq, Hq, float(k_scale),
+                                     float(v_scale), float(sm_scale), rp, nr, _p(out), _p(lse))
+    if rc:
+        raise ValueError(f"oracle prefill attention failed ({rc})")
     return out, lse
 
 

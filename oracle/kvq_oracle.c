@@ -468,6 +468,52 @@ int orc_decode_attention(int fmt, const uint16_t* q, const void* k_cache, const 
 }
 
 /*
+ * Chunked-prefill attention: the Tq newest tokens of each sequence, already
+ * written to the cache, attend causally to the cache.  Long prompts are fed
+ * in chunks of a fixed token budget with the earlier prefix reused from the
+ * cache ("Dual R9700 model and spec-decode campaign", fixed knobs:
+ * long-prefill-token-threshold 2048 with prefix caching; "FP8 KV calibration
+ * guide", first paragraph: TTFT at ~126k context with FP8 KV).
+ *   Sequence b holds len_b = seq_lens[b] tokens; its query token i
+ *   (0 <= i < Tq) sits at position p = len_b - Tq + i and attends to the
+ *   cache tokens [0, p] (itself included), with the same scores, softmax and
+ *   GQA mapping as a decode query.  A query with p < 0 (a sequence shorter
+ *   than the chunk) attends to nothing: out = 0, lse = -inf.
+ * q is [B][Tq][Hq][D] BF16; out is [B][Tq][Hq][D] and lse [B][Tq][Hq]
+ * (float64).  If rows is non-NULL only the n_rows (b, i, j) triples listed in
+ * it (rows[3r], rows[3r + 1], rows[3r + 2]) are computed; other outputs are
+ * left untouched.
+ */
+int orc_prefill_attention(int fmt, const uint16_t* q, const void* k_cache, const void* v_cache,
+                          int64_t num_blocks, int H, int D, const int32_t* block_table,
+                          int max_blocks, const int32_t* seq_lens, int B, int Tq, int Hq,
+                          float k_scale, float v_scale, double sm_scale, const int32_t* rows,
+                          int64_t n_rows, double* out, double* lse) {
+  int G = Hq / H;
+  int64_t total = rows ? n_rows : (int64_t)B * Tq * Hq;
+  for (int64_t r = 0; r < total; r++) {
+    int b = rows ? rows[3 * r] : (int)(r / ((int64_t)Tq * Hq));
+    int i = rows ? rows[3 * r + 1] : (int)((r / Hq) % Tq);
+    int j = rows ? rows[3 * r + 2] : (int)(r % Hq);
+    int64_t row = ((int64_t)b * Tq + i) * Hq + j;
+    int64_t p = (int64_t)seq_lens[b] - Tq + i;
+    double m, l;
+    double* o = out + row * D;
+    int rc = orc_attention_range(fmt, q + row * D, k_cache, v_cache, num_blocks, H, D,
+                                 block_table + (int64_t)b * max_blocks, j / G, 0, p + 1, k_scale,
+                                 v_scale, sm_scale, o, &m, &l);
+    if (rc) return rc;
+    if (l > 0.0) {
+      for (int d = 0; d < D; d++) o[d] /= l;
+      lse[row] = m + log(l);
+    } else {
+      lse[row] = -INFINITY;
+    }
+  }
+  return 0;
+}
+
+/*
  * Merge of n partial results (o_unnorm_i, m_i, l_i) of disjoint context
  * ranges into the full one:
  *   M = max_i m_i,  L = sum_i exp(m_i - M) l_i,
