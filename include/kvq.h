@@ -234,6 +234,41 @@ kvq_status kv_decode_workspace_size_window(int32_t fmt, int32_t num_seqs, int32_
                                            int32_t max_seq_len, int32_t window,
                                            int32_t num_splits, size_t* bytes);
 
+/* Chunked-prefill attention over the paged cache: the attention of a prompt
+ * chunk's own tokens, after kv_quantize_write has put them in the cache.
+ * Long prompts are fed in chunks of a fixed token budget that attend to the
+ * prefix already cached ("Dual R9700 model and spec-decode campaign", fixed
+ * knobs: long-prefill-token-threshold 2048 with prefix caching; "FP8 KV
+ * calibration guide", first paragraph: TTFT at ~126k context with FP8 KV).
+ *   q          [num_seqs][num_q_tokens][num_q_heads][head_dim] BF16: the
+ *              num_q_tokens newest tokens of each sequence.  Device, 16-byte
+ *              aligned.
+ *   seq_lens   [num_seqs] int32: cached tokens of each sequence, the chunk
+ *              included.  Query i of sequence b sits at position
+ *              p = seq_lens[b] - num_q_tokens + i and attends to the cache
+ *              tokens [0, p] (causal, itself included); a query with p < 0
+ *              attends to nothing (out = 0, lse = -inf).
+ *   block_table, max_blocks, cache, d_k_scale, d_v_scale, sm_scale: as for
+ *              kv_decode_attention (GQA: query head j reads KV head
+ *              j / (num_q_heads / num_kv_heads)).
+ *   out        [num_seqs][num_q_tokens][num_q_heads][head_dim] fp32, 16-byte
+ *              aligned; lse [num_seqs][num_q_tokens][num_q_heads] fp32 (natural
+ *              log of the scaled scores) or NULL.
+ * Scores, softmax and dequantisation are those of kv_decode_attention; the
+ * result matches float64 attention over the dequantised cache within the same
+ * tolerances.  No workspace.  num_q_heads / num_kv_heads must be at most 128
+ * (KVQ_ERR_UNSUPPORTED otherwise).  Device-side problems set d_err bits as in
+ * kv_decode_attention: a bad block id (its page's keys are skipped), a
+ * seq_lens entry outside [0, max_blocks * 16] (that sequence's outputs are
+ * empty), a bad scale (all outputs empty).  Asynchronous on `stream`;
+ * ordinary stream ordering (no early start behind a write). */
+kvq_status kv_prefill_attention(int32_t fmt, const void* q, const kvq_cache* cache,
+                                const int32_t* block_table, int32_t max_blocks,
+                                const int32_t* seq_lens, int32_t num_seqs, int32_t num_q_tokens,
+                                int32_t num_q_heads, const float* d_k_scale,
+                                const float* d_v_scale, float sm_scale, float* out, float* lse,
+                                int32_t* d_err, kvq_stream stream);
+
 /* kv_decode_attention without a caller workspace, for callers that cannot
  * allocate device memory when they run a decode step (their device memory
  * belongs to a fixed pool they must not bypass, they may not pay a

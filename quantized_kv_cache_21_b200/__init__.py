@@ -32,7 +32,8 @@ DERR_TIMEOUT = 0x10
 EXPORTS = ("kvq_status_string", "kvq_last_error", "kv_cache_bytes", "kv_scale_from_absmax",
            "kv_scale_from_absmax_device", "kv_calibrate_absmax", "kv_quantize_write",
            "kv_decode_workspace_size", "kv_decode_attention", "kv_decode_attention_static_ws",
-           "kv_decode_attention_window", "kv_decode_workspace_size_window", "kv_dequantize")
+           "kv_decode_attention_window", "kv_decode_workspace_size_window",
+           "kv_prefill_attention", "kv_dequantize")
 
 
 class KvqError(RuntimeError):
@@ -77,6 +78,8 @@ def lib() -> ctypes.CDLL:
                                            f32, P, P, P, sz, P, P],
             "kv_decode_workspace_size_window": [i32, i32, i32, i32, i32, i32, i32, i32,
                                                 ctypes.POINTER(sz)],
+            "kv_prefill_attention": [i32, P, CP, P, i32, P, i32, i32, i32, P, P, f32, P, P, P,
+                                     P],
             "kv_dequantize": [i32, CP, P, i64, P, P, P, P, P, P],
         }
         for name, args in sigs.items():
@@ -255,6 +258,23 @@ def kv_decode_attention_window(fmt, q: torch.Tensor, cache: KVCache, block_table
                                             _ptr(v_scale), float(sm_scale), _ptr(out), _ptr(lse),
                                             _ptr(workspace), ws_bytes, _ptr(d_err),
                                             _stream(stream)))
+
+
+def kv_prefill_attention(fmt, q: torch.Tensor, cache: KVCache, block_table: torch.Tensor,
+                         seq_lens: torch.Tensor, k_scale, v_scale, out: torch.Tensor,
+                         lse: torch.Tensor | None, d_err: torch.Tensor | None = None,
+                         sm_scale: float = 0.0, stream=None):
+    """Chunked-prefill attention (see include/kvq.h).  q: BF16 [B][Tq][Hq][D],
+    the Tq newest tokens of each sequence, already in the cache; seq_lens int32
+    [B] counts them; out fp32 [B][Tq][Hq][D]; lse fp32 [B][Tq][Hq] or None."""
+    assert q.dtype == torch.bfloat16 and q.is_contiguous() and q.dim() == 4
+    assert block_table.dtype == torch.int32 and seq_lens.dtype == torch.int32
+    assert out.dtype == torch.float32 and out.is_contiguous()
+    B, Tq, Hq, _ = q.shape
+    _check(lib().kv_prefill_attention(_fmt(fmt), _ptr(q), cache.c, _ptr(block_table),
+                                      block_table.shape[1], _ptr(seq_lens), B, Tq, Hq,
+                                      _ptr(k_scale), _ptr(v_scale), float(sm_scale), _ptr(out),
+                                      _ptr(lse), _ptr(d_err), _stream(stream)))
 
 
 def kv_dequantize(fmt, cache: KVCache, slots: torch.Tensor, k_scale, v_scale,

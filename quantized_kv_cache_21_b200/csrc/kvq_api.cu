@@ -466,6 +466,63 @@ kvq_status kv_decode_attention_window(int32_t fmt, const void* q, const kvq_cach
   return e == cudaSuccess ? KVQ_OK : cuda_fail(e, "decode kernel");
 }
 
+kvq_status kv_prefill_attention(int32_t fmt, const void* q, const kvq_cache* cache,
+                                const int32_t* block_table, int32_t max_blocks,
+                                const int32_t* seq_lens, int32_t num_seqs, int32_t num_q_tokens,
+                                int32_t num_q_heads, const float* d_k_scale,
+                                const float* d_v_scale, float sm_scale, float* out, float* lse,
+                                int32_t* d_err, kvq_stream stream) {
+  kvq_status s = check_cache(fmt, cache);
+  if (s != KVQ_OK) return s;
+  const int D = cache->head_dim, Hkv = cache->num_kv_heads;
+  if (num_seqs < 0 || num_q_tokens < 0)
+    return fail(KVQ_ERR_INVALID_ARG, "num_seqs %d / num_q_tokens %d", num_seqs, num_q_tokens);
+  if (num_q_heads < 1 || num_q_heads % Hkv != 0)
+    return fail(KVQ_ERR_INVALID_ARG, "num_q_heads %d not a multiple of num_kv_heads %d",
+                num_q_heads, Hkv);
+  const int G = num_q_heads / Hkv;
+  if (G > kvq::prefill_rows())
+    return fail(KVQ_ERR_UNSUPPORTED, "%d query heads per KV head (at most %d)", G,
+                kvq::prefill_rows());
+  if (num_seqs == 0 || num_q_tokens == 0) return KVQ_OK;
+  if (!q || !aligned(q, 16)) return fail(KVQ_ERR_INVALID_ARG, "q NULL or not 16-byte aligned");
+  if (!out || !aligned(out, 16)) return fail(KVQ_ERR_INVALID_ARG, "out NULL or not 16-byte aligned");
+  if (!block_table || !seq_lens) return fail(KVQ_ERR_INVALID_ARG, "block_table/seq_lens NULL");
+  if (max_blocks < 1) return fail(KVQ_ERR_INVALID_ARG, "max_blocks %d", max_blocks);
+  if (fmt != KVQ_FMT_BF16 && (!d_k_scale || !d_v_scale))
+    return fail(KVQ_ERR_INVALID_ARG, "quantized formats need d_k_scale and d_v_scale");
+  if (sm_scale == 0.0f) sm_scale = 1.0f / sqrtf((float)D);
+  if (!isfinite(sm_scale)) return fail(KVQ_ERR_INVALID_ARG, "sm_scale not finite");
+  s = check_device();
+  if (s != KVQ_OK) return s;
+  kvq::PrefillParams p;
+  p.q = static_cast<const uint16_t*>(q);
+  p.block_table = block_table;
+  p.seq_lens = seq_lens;
+  p.kc = static_cast<const uint8_t*>(cache->k);
+  p.vc = static_cast<const uint8_t*>(cache->v);
+  p.k_scale = d_k_scale;
+  p.v_scale = d_v_scale;
+  p.out = out;
+  p.lse = lse;
+  p.d_err = d_err;
+  p.num_blocks = cache->num_blocks;
+  p.max_blocks = max_blocks;
+  p.B = num_seqs;
+  p.Tq = num_q_tokens;
+  p.Hq = num_q_heads;
+  p.Hkv = Hkv;
+  p.G = G;
+  p.QT = kvq::prefill_rows() / G;
+  p.n_qblk = (num_q_tokens + p.QT - 1) / p.QT;
+  p.sm_scale = sm_scale;
+  const int64_t ctas = static_cast<int64_t>(p.n_qblk) * Hkv * num_seqs;
+  if (ctas > 0x7fffffffLL) return fail(KVQ_ERR_INVALID_ARG, "problem too large (%lld CTAs)",
+                                       (long long)ctas);
+  cudaError_t e = kvq::launch_prefill(fmt, D, p, ctas, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? KVQ_OK : cuda_fail(e, "prefill kernel");
+}
+
 kvq_status kv_dequantize(int32_t fmt, const kvq_cache* cache, const int64_t* slots, int64_t n,
                          const float* d_k_scale, const float* d_v_scale, float* k_out,
                          float* v_out, int32_t* d_err, kvq_stream stream) {

@@ -44,6 +44,30 @@ bool decode_config(int fmt, int D, DecodeConfig* cfg);
 cudaError_t launch_decode(int fmt, int D, const CUtensorMap* maps, const DecodeParams& p,
                           int ctas, cudaStream_t stream);
 
+struct PrefillParams {
+  const uint16_t* q;          // [B][Tq][Hq][D] bf16: the Tq newest tokens of each sequence
+  const int32_t* block_table; // [B][max_blocks]
+  const int32_t* seq_lens;    // [B], cached tokens including the chunk
+  const uint8_t* kc;          // cache pages [num_blocks][Hkv][head page]
+  const uint8_t* vc;
+  const float* k_scale;       // device scalar (FP8: s, NVFP4: g); unused for BF16
+  const float* v_scale;
+  float* out;                 // [B][Tq][Hq][D]
+  float* lse;                 // [B][Tq][Hq] or null
+  int* d_err;
+  int64_t num_blocks;
+  int max_blocks;
+  int B, Tq, Hq, Hkv, G;
+  int QT;                     // query tokens per CTA (rows per CTA / G)
+  int n_qblk;                 // ceil(Tq / QT)
+  float sm_scale;
+};
+
+// Rows ((query token, query head) pairs of one KV head) per prefill CTA.
+int prefill_rows();
+cudaError_t launch_prefill(int fmt, int D, const PrefillParams& p, int64_t ctas,
+                           cudaStream_t stream);
+
 struct QuantParams {
   const uint16_t* k;
   const uint16_t* v;

@@ -1,13 +1,14 @@
-"""Run a few decode launches of one scenario (for profilers and quick checks).
+"""Run a few decode (or chunked-prefill) launches of one scenario (for profilers).
 
     python -m quantized_kv_cache_21_b200.run_decode --workload agents-fp8-4x127k \
         --fmt nvfp4 --seq-len 32768 --launches 4
 
 Builds the named workload's cache (optionally with another format, context
 length, batch or head_dim), writes the step's tokens with kv_quantize_write,
-then launches kv_decode_attention --launches times
-on the current stream and prints the device error word and the KV-scan bytes
-of one launch.  Nothing is timed here: bench.py owns timing."""
+then launches kv_decode_attention (with --prefill: kv_prefill_attention of the
+step's chunk of new tokens) --launches times on the current stream and prints
+the device error word and the KV-scan bytes (prefill: algorithmic FLOPs) of one
+launch.  Nothing is timed here: bench.py owns timing."""
 from __future__ import annotations
 
 import argparse
@@ -27,6 +28,8 @@ def main(argv=None) -> int:
     ap.add_argument("--batch", type=int, default=None)
     ap.add_argument("--head-dim", type=int, choices=[64, 128], default=None)
     ap.add_argument("--launches", type=int, default=4)
+    ap.add_argument("--prefill", action="store_true",
+                    help="launch the chunk's prefill attention instead of the decode")
     args = ap.parse_args(argv)
     w = wl.WORKLOADS[args.workload]
     over = {}
@@ -39,11 +42,15 @@ def main(argv=None) -> int:
     w = dataclasses.replace(w, **over) if over else w
     sc = DecodeScenario(w, fmt=args.fmt or w.fmt)
     sc.write()  # the step's own tokens, so the scanned cache is complete
+    if args.prefill:
+        sc.prefill_setup()
     for _ in range(args.launches):
-        sc.decode()
+        sc.prefill() if args.prefill else sc.decode()
     torch.cuda.synchronize()
+    what = (f"prefill chunk {sc.chunk}, FLOPs per launch {sc.prefill_flops}" if args.prefill
+            else f"KV-scan bytes per launch {sc.scan_bytes}")
     print(f"workload {w.name} fmt {sc.fmt} B {sc.B} L {sc.L} D {sc.D}: "
-          f"device error word {int(sc.err.item())}, KV-scan bytes per launch {sc.scan_bytes}")
+          f"device error word {int(sc.err.item())}, {what}")
     return 0 if int(sc.err.item()) == 0 else 1
 
 

@@ -146,3 +146,32 @@ class DecodeScenario:
     def step(self, stream=None):
         self.write(stream)
         self.decode(stream)
+
+    # ---- chunked prefill: the step's chunk of new tokens attends to the cache
+    def prefill_setup(self):
+        """Seeded BF16 queries of the step's chunk ([B][chunk][Hq][D]) and their
+        output buffers (created on first use)."""
+        if hasattr(self, "q_chunk"):
+            return
+        B, Hq, D, dev = self.B, self.Hq, self.D, self.device
+        g = torch.Generator(device=dev)
+        g.manual_seed(self.w.seed * 7919 + 29 + self.seq_offset)
+        self.q_chunk = torch.randn((B, self.chunk, Hq, D), generator=g,
+                                   device=dev).to(torch.bfloat16)
+        self.out_chunk = torch.empty((B, self.chunk, Hq, D), dtype=torch.float32, device=dev)
+        self.lse_chunk = torch.empty((B, self.chunk, Hq), dtype=torch.float32, device=dev)
+
+    def prefill(self, stream=None):
+        """Attention of the chunk's queries over the cache (after write())."""
+        kvq.kv_prefill_attention(self.fmt, self.q_chunk, self.cache, self.d_bt, self.d_lens,
+                                 self.d_ks, self.d_vs, self.out_chunk, self.lse_chunk, self.err,
+                                 stream=stream)
+
+    @property
+    def prefill_flops(self) -> int:
+        """Algorithmic FLOPs of the chunk prefill: 2 D (QK) + 2 D (PV) per
+        (query row, attended key); query i of a chunk of T at the end of a
+        sequence of length n attends to n - T + i + 1 keys."""
+        T, D, Hq = self.chunk, self.D, self.Hq
+        keys = sum(T * (int(n) - T) + T * (T + 1) // 2 for n in self.lens)
+        return 4 * D * Hq * keys
