@@ -318,6 +318,13 @@ __global__ void __launch_bounds__(kThreads, 2) kvq_prefill_kernel(const PrefillP
   const int npages = (n_keys + kPage - 1) / kPage;
   const int nblk = (n_keys + kKeys - 1) / kKeys;
 
+  // Scores are scaled by c = sm_scale * k_scale * log2(e) after the running max
+  // of the raw ones is taken, so c must not be negative: a negative sm_scale is
+  // moved into Q's sign (exact).  c = 0 (an all-zero NVFP4 K tensor, whose
+  // scores are all 0) becomes a tiny positive c with the same result.
+  const float c_log2 = p.sm_scale * ks * kLog2e;
+  const uint32_t q_sign = c_log2 < 0.f ? 0x80008000u : 0u;
+  const float c_abs = fmaxf(fabsf(c_log2), 1e-30f);
   // Q row -> sQ (K-major A tile: [D/64][128 rows][128 B])
   {
     const uint4* qrow = reinterpret_cast<const uint4*>(
@@ -331,6 +338,10 @@ __global__ void __launch_bounds__(kThreads, 2) kvq_prefill_kernel(const PrefillP
         w.z = pack_f16x2(bf16_lo(w.z), bf16_hi(w.z));
         w.w = pack_f16x2(bf16_lo(w.w), bf16_hi(w.w));
       }
+      w.x ^= q_sign;
+      w.y ^= q_sign;
+      w.z ^= q_sign;
+      w.w ^= q_sign;
       *reinterpret_cast<uint4*>(sQ + (c >> 3) * 16384 + sw128(tid, c & 7)) = w;
     }
   }
@@ -352,7 +363,6 @@ __global__ void __launch_bounds__(kThreads, 2) kvq_prefill_kernel(const PrefillP
   const uint32_t tm = s_tmem;
   const uint32_t tm_row = tm + (static_cast<uint32_t>(warp * 32) << 16);
 
-  const float c_log2 = p.sm_scale * ks * kLog2e;
   float m_ref = -kInf, l = 0.f;
   uint32_t ph = 0;
   bool failed = false;
@@ -379,17 +389,21 @@ __global__ void __launch_bounds__(kThreads, 2) kvq_prefill_kernel(const PrefillP
     tmem_ld32(tm_row + kColS + 32, sv + 32);
     tmem_wait_ld();
 
-    // ---- scale, mask, lazy running max
+    // ---- mask, lazy running max (scores stay raw; c_abs > 0 scales them)
     const bool any_bad = s_bad[0] | s_bad[1] | s_bad[2] | s_bad[3];
-    const bool need_mask = key0 + kKeys - 1 > pos || any_bad;
-    float mx = -kInf;
+    if (key0 + kKeys - 1 > pos || any_bad) {
 #pragma unroll
-    for (int k = 0; k < kKeys; ++k) {
-      float v = sv[k] * c_log2;
-      if (need_mask && (key0 + k > pos || s_bad[k >> 4])) v = -kInf;
-      sv[k] = v;
-      mx = fmaxf(mx, v);
+      for (int k = 0; k < kKeys; ++k)
+        if (key0 + k > pos || s_bad[k >> 4]) sv[k] = -kInf;
     }
+    float t[32];  // max as a tree: depth 6 instead of a chain of 64
+#pragma unroll
+    for (int i = 0; i < 32; ++i) t[i] = fmaxf(sv[i], sv[i + 32]);
+#pragma unroll
+    for (int w = 16; w >= 1; w >>= 1)
+#pragma unroll
+      for (int i = 0; i < w; ++i) t[i] = fmaxf(t[i], t[i + w]);
+    const float mx = t[0] * c_abs;
     float m_new = m_ref;
     if (mx > m_ref + kGap || (m_ref == -kInf && mx > -kInf)) m_new = mx;
     const bool resc = m_new != m_ref && m_ref != -kInf;
@@ -407,20 +421,22 @@ __global__ void __launch_bounds__(kThreads, 2) kvq_prefill_kernel(const PrefillP
       tmem_wait_st();
     }
     m_ref = m_new;
-    float ps = 0.f;
+    // p = 2^(s c - m); a row with nothing unmasked yet has s = -inf throughout
+    const float neg_m = m_ref == -kInf ? 0.f : -m_ref;
+    float ps8[8];
 #pragma unroll
     for (int c = 0; c < 8; ++c) {  // keys 8c .. 8c + 7
       uint32_t hi[4], lo[4];
+      float pc[8];
 #pragma unroll
-      for (int x = 0; x < 4; ++x) {
-        const float p0 = m_ref == -kInf ? 0.f : fast_exp2(sv[8 * c + 2 * x] - m_ref);
-        const float p1 = m_ref == -kInf ? 0.f : fast_exp2(sv[8 * c + 2 * x + 1] - m_ref);
-        ps += p0 + p1;
-        split_pair<FMT>(p0, p1, hi[x], lo[x]);
-      }
+      for (int x = 0; x < 8; ++x) pc[x] = fast_exp2(fmaf(sv[8 * c + x], c_abs, neg_m));
+#pragma unroll
+      for (int x = 0; x < 4; ++x) split_pair<FMT>(pc[2 * x], pc[2 * x + 1], hi[x], lo[x]);
+      ps8[c] = ((pc[0] + pc[1]) + (pc[2] + pc[3])) + ((pc[4] + pc[5]) + (pc[6] + pc[7]));
       *reinterpret_cast<uint4*>(sPh + sw128(tid, c)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
       *reinterpret_cast<uint4*>(sPl + sw128(tid, c)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
     }
+    const float ps = ((ps8[0] + ps8[1]) + (ps8[2] + ps8[3])) + ((ps8[4] + ps8[5]) + (ps8[6] + ps8[7]));
     l = l * alpha + ps;
     fence_proxy_async_smem();
     tc_fence_before();

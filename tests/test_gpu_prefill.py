@@ -90,8 +90,9 @@ def test_chunk_of_one_token_is_the_decode():
 def test_sm_scale_and_no_lse():
     c = Case("nvfp4", 2, 1, 8, 64, [70, 33], seed=7300)
     q = chunk_q(c, 17, 7301)
-    out, lse = run(c, q, sm_scale=0.3)
-    assert_attention_close(out, lse, *reference(c, q, sm_scale=0.3))
+    for sm in (-0.2, 0.3):  # a negative scale flips which key dominates
+        out, lse = run(c, q, sm_scale=sm)
+        assert_attention_close(out, lse, *reference(c, q, sm_scale=sm))
     out2 = torch.full(q.shape, float("nan"), device=DEV)
     kvq.kv_prefill_attention("nvfp4", to_dev_bits(q), c.cache, c.d_bt, c.d_lens, c.d_ks, c.d_vs,
                              out2, None, c.err, 0.3)
