@@ -530,8 +530,9 @@ def main():
             "ms_per_launch": t_pf * 1e3, "algorithmic_flops": s3.prefill_flops,
             "TFLOPs": tf, "peak_TFLOPs": pk_s, "peak": f"{pk_kind} bf16 dense, sustained",
             "frac_of_tensor_peak": tf / pk_s, "frac_of_burst_peak": tf / pk_b,
-            "mma": "mma.sync m16n8k16 (f16; bf16 for BF16 pages), fp32 accumulate; P enters PV "
-                   "as two 16-bit halves (executed MMA flops = 1.5x algorithmic)"}
+            "mma": "tcgen05.mma kind::f16 (bf16 for BF16 pages), M=128, fp32 accumulators in "
+                   "tensor memory; P enters PV as two 16-bit halves (executed MMA flops = 1.5x "
+                   "algorithmic)"}
         del s3
         torch.cuda.empty_cache()
 
