@@ -70,3 +70,29 @@ def test_host_scale_matches_oracle_bit_exact(L):
     for bad in (-1.0, float("nan"), float("inf")):
         with pytest.raises(kvq.KvqError):
             kvq.kv_scale_from_absmax("fp8", bad)
+
+
+def test_prefill_argument_checks_run_on_the_host(L):
+    """kv_prefill_attention validates its arguments before touching the device:
+    these calls return their status codes on a machine without a GPU (the cache
+    pointers are never dereferenced)."""
+    fake = 1 << 20  # 256-byte aligned, never dereferenced
+    cache = kvq._Cache(kvq.FORMATS["fp8"], 16, 8, 2, 64, fake, fake)
+    cp = ctypes.byref(cache)
+
+    def call(B=1, Tq=4, Hq=8, q=fake, out=fake, bt=fake, lens=fake, ks=fake, vs=fake, fmt=1):
+        return L.kv_prefill_attention(fmt, q, cp, bt, 4, lens, B, Tq, Hq, ks, vs, 0.0, out, None,
+                                      None, None)
+
+    assert call(Hq=3) == 1                  # not a multiple of the 2 KV heads
+    assert call(Hq=2 * 129) == 2            # 129 query heads per KV head
+    assert call(B=-1) == 1
+    assert call(Tq=-1) == 1
+    assert call(Tq=0) == 0                  # an empty chunk launches nothing
+    assert call(B=0) == 0
+    assert call(q=None) == 1
+    assert call(q=fake + 8) == 1            # q not 16-byte aligned
+    assert call(out=fake + 4) == 1
+    assert call(bt=None) == 1
+    assert call(ks=None) == 1               # quantized formats need both scales
+    assert call(fmt=2) == 1                 # cache format differs from fmt
