@@ -29,9 +29,11 @@
 //      lazily: the reference max moves only when a score exceeds it by more
 //      than 2^8, and only then is its row of O (in tensor memory) rescaled, so
 //      P stays <= 256;
-//   5. P is written to shared memory as a 16-bit high part and its residual
-//      (two K-major A tiles), and one thread issues O += P_hi V + P_lo V
-//      (M 128, N = head_dim, K 64; V read MN-major straight from its tile);
+//   5. P is written back over the row's S in tensor memory as a 16-bit high
+//      part and its residual (two K-major A operands, two 16-bit values per
+//      column), and one thread issues O += P_hi V + P_lo V with A read from
+//      tensor memory (M 128, N = head_dim, K 64; V read MN-major straight
+//      from its tile);
 //   6. while that runs, the next block's K is decoded into its tile; after the
 //      PV commit, V.
 // Q is staged once.  Online softmax in the exp2 domain; the per-layer K scale
@@ -78,6 +80,17 @@ __device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t a, uint64_t b, 
       " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n}\n" ::"r"(
           d_tmem),
       "l"(a), "l"(b), "r"(idesc), "r"(acc), "r"(0u), "r"(0u), "r"(0u), "r"(0u)
+      : "memory");
+}
+// D[tmem] (+)= A[tmem] * B[smem]: A (K-major, 16-bit elements packed two per
+// 32-bit column, row i in lane i) read from tensor memory.
+__device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b,
+                                          uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, {%5, %6, %7, %8}, p;\n}\n" ::"r"(
+          d_tmem),
+      "r"(a_tmem), "l"(b), "r"(idesc), "r"(acc), "r"(0u), "r"(0u), "r"(0u), "r"(0u)
       : "memory");
 }
 // Arrive once on bar when every MMA this thread issued so far has completed.
@@ -250,9 +263,9 @@ __host__ __device__ constexpr uint32_t tmem_cols() {
 }
 template <int D>
 constexpr size_t smem_bytes() {
-  // Q [D/64][128][128 B], K and V [D/64][64][128 B], P hi and lo [128][128 B],
-  // plus 1 KB to align the tiles to the 1024-byte swizzle repeat
-  return (D / 64) * (16384 + 2 * 8192) + 2 * 16384 + 1024;
+  // Q [D/64][128][128 B], K and V [D/64][64][128 B], plus 1 KB to align the
+  // tiles to the 1024-byte swizzle repeat (P lives in tensor memory)
+  return (D / 64) * (16384 + 2 * 8192) + 1024;
 }
 
 template <int FMT, int D>
@@ -268,8 +281,6 @@ __global__ void __launch_bounds__(kThreads, 2) kvq_prefill_kernel(const PrefillP
                                            ~static_cast<uintptr_t>(1023));
   uint8_t* sK = sQ + KA * 16384;
   uint8_t* sV = sK + KA * 8192;
-  uint8_t* sPh = sV + KA * 8192;
-  uint8_t* sPl = sPh + 16384;
   __shared__ uint64_t bar_s, bar_o;
   __shared__ uint32_t s_tmem;
   __shared__ int s_bad[4];
@@ -423,22 +434,25 @@ __global__ void __launch_bounds__(kThreads, 2) kvq_prefill_kernel(const PrefillP
     m_ref = m_new;
     // p = 2^(s c - m); a row with nothing unmasked yet has s = -inf throughout
     const float neg_m = m_ref == -kInf ? 0.f : -m_ref;
+    // P's two 16-bit halves replace this row's S in tensor memory (S is in
+    // registers now): columns [S, S + 32) high parts, [S + 32, S + 64) residuals
     float ps8[8];
+    uint32_t phi[32], plo[32];
 #pragma unroll
     for (int c = 0; c < 8; ++c) {  // keys 8c .. 8c + 7
-      uint32_t hi[4], lo[4];
       float pc[8];
 #pragma unroll
       for (int x = 0; x < 8; ++x) pc[x] = fast_exp2(fmaf(sv[8 * c + x], c_abs, neg_m));
 #pragma unroll
-      for (int x = 0; x < 4; ++x) split_pair<FMT>(pc[2 * x], pc[2 * x + 1], hi[x], lo[x]);
+      for (int x = 0; x < 4; ++x)
+        split_pair<FMT>(pc[2 * x], pc[2 * x + 1], phi[4 * c + x], plo[4 * c + x]);
       ps8[c] = ((pc[0] + pc[1]) + (pc[2] + pc[3])) + ((pc[4] + pc[5]) + (pc[6] + pc[7]));
-      *reinterpret_cast<uint4*>(sPh + sw128(tid, c)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-      *reinterpret_cast<uint4*>(sPl + sw128(tid, c)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
     }
+    tmem_st32(tm_row + kColS, reinterpret_cast<const float*>(phi));
+    tmem_st32(tm_row + kColS + 32, reinterpret_cast<const float*>(plo));
     const float ps = ((ps8[0] + ps8[1]) + (ps8[2] + ps8[3])) + ((ps8[4] + ps8[5]) + (ps8[6] + ps8[7]));
     l = l * alpha + ps;
-    fence_proxy_async_smem();
+    tmem_wait_st();
     tc_fence_before();
     __syncthreads();
 
@@ -446,10 +460,10 @@ __global__ void __launch_bounds__(kThreads, 2) kvq_prefill_kernel(const PrefillP
     if (tid == 0) {
       tc_fence_after();
 #pragma unroll
-      for (int s = 0; s < kKeys / 16; ++s) {
+      for (int s = 0; s < kKeys / 16; ++s) {  // 16 keys = 8 columns of packed P
         const uint64_t bv = sdesc(sV + s * 2048, kKeys * 128, 1024);
-        tc_mma(tm + kColO, sdesc(sPh + s * 32, 16, 1024), bv, kIdPV, kb > 0 || s > 0);
-        tc_mma(tm + kColO, sdesc(sPl + s * 32, 16, 1024), bv, kIdPV, 1u);
+        tc_mma_ts(tm + kColO, tm + kColS + 8 * s, bv, kIdPV, kb > 0 || s > 0);
+        tc_mma_ts(tm + kColO, tm + kColS + 32 + 8 * s, bv, kIdPV, 1u);
       }
       tc_commit(&bar_o);
     }
