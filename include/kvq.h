@@ -269,6 +269,15 @@ kvq_status kv_prefill_attention(int32_t fmt, const void* q, const kvq_cache* cac
                                 const float* d_v_scale, float sm_scale, float* out, float* lse,
                                 int32_t* d_err, kvq_stream stream);
 
+/* Self-test of the bounded wait behind every mbarrier wait in the library's
+ * kernels (no attention computed).  One warp waits on an mbarrier phase:
+ * with arrive != 0 the phase is completed first and the wait succeeds; with
+ * arrive = 0 nothing completes it, the wait gives up after about two seconds
+ * and KVQ_DERR_TIMEOUT is set in *d_err (device int32, caller-zeroed).  The
+ * context stays usable either way.  KVQ_ERR_INVALID_ARG if d_err is NULL.
+ * Asynchronous on `stream`. */
+kvq_status kvq_selftest_bounded_wait(int32_t* d_err, int32_t arrive, kvq_stream stream);
+
 /* kv_decode_attention without a caller workspace, for callers that cannot
  * allocate device memory when they run a decode step (their device memory
  * belongs to a fixed pool they must not bypass, they may not pay a

@@ -33,7 +33,7 @@ EXPORTS = ("kvq_status_string", "kvq_last_error", "kv_cache_bytes", "kv_scale_fr
            "kv_scale_from_absmax_device", "kv_calibrate_absmax", "kv_quantize_write",
            "kv_decode_workspace_size", "kv_decode_attention", "kv_decode_attention_static_ws",
            "kv_decode_attention_window", "kv_decode_workspace_size_window",
-           "kv_prefill_attention", "kv_dequantize")
+           "kv_prefill_attention", "kv_dequantize", "kvq_selftest_bounded_wait")
 
 
 class KvqError(RuntimeError):
@@ -81,6 +81,7 @@ def lib() -> ctypes.CDLL:
             "kv_prefill_attention": [i32, P, CP, P, i32, P, i32, i32, i32, P, P, f32, P, P, P,
                                      P],
             "kv_dequantize": [i32, CP, P, i64, P, P, P, P, P, P],
+            "kvq_selftest_bounded_wait": [P, i32, P],
         }
         for name, args in sigs.items():
             fn = getattr(L, name)
@@ -284,3 +285,10 @@ def kv_dequantize(fmt, cache: KVCache, slots: torch.Tensor, k_scale, v_scale,
     _check(lib().kv_dequantize(_fmt(fmt), cache.c, _ptr(slots), slots.numel(), _ptr(k_scale),
                                _ptr(v_scale), _ptr(k_out), _ptr(v_out), _ptr(d_err),
                                _stream(stream)))
+
+
+def kvq_selftest_bounded_wait(d_err: torch.Tensor, arrive: bool, stream=None):
+    """Run the bounded-wait self-test (see include/kvq.h): arrive=False makes
+    the wait run out (about 2 s) and set DERR_TIMEOUT in d_err."""
+    assert d_err.dtype == torch.int32
+    _check(lib().kvq_selftest_bounded_wait(_ptr(d_err), int(bool(arrive)), _stream(stream)))

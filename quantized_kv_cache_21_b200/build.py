@@ -16,7 +16,8 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libkvq.so")
-SOURCES = ["kvq_api.cu", "kvq_decode.cu", "kvq_prefill.cu", "kvq_quant.cu", "kvq_static_ws.cu"]
+SOURCES = ["kvq_api.cu", "kvq_decode.cu", "kvq_prefill.cu", "kvq_quant.cu", "kvq_selftest.cu",
+           "kvq_static_ws.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

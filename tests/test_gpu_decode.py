@@ -217,3 +217,26 @@ def test_decode_launched_right_after_a_write(fmt, D):
     torch.cuda.synchronize()
     assert int(c.err.item()) == 0
     assert_attention_close(out.cpu().numpy(), lse.cpu().numpy(), *c.reference())
+
+
+def test_bounded_wait_times_out_and_reports():
+    """The bounded mbarrier wait behind every kernel's waits: a completed phase
+    passes with no error; a phase nothing completes gives up after about two
+    seconds with DERR_TIMEOUT in the error word, and the context stays usable
+    (a decode right after it matches the oracle)."""
+    import time
+
+    err = new_err()
+    kvq.kvq_selftest_bounded_wait(err, True)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    t0 = time.monotonic()
+    kvq.kvq_selftest_bounded_wait(err, False)
+    torch.cuda.synchronize()
+    dt = time.monotonic() - t0
+    assert int(err.item()) == kvq.DERR_TIMEOUT
+    assert 1.0 < dt < 20.0, f"wait gave up after {dt:.2f} s"
+    c = Case("fp8", 2, 2, 16, 128, [300, 77], seed=7700)
+    out, lse = c.decode()
+    assert int(c.err.item()) == 0
+    assert_attention_close(out, lse, *c.reference())
