@@ -24,6 +24,23 @@ def kv_scan_bytes(fmt: str, lens, H: int, D: int) -> int:
     return int(round(sum(int(n) for n in lens) * H * 2 * D * BYTES_PER_ELEM[fmt]))
 
 
+def prefill_flops(lens, chunk: int, Hq: int, D: int) -> int:
+    """Algorithmic FLOPs of a chunked prefill: 2 D (QK) + 2 D (PV) per (query
+    row, attended key).  The chunk is the last `chunk` tokens of each sequence;
+    query i of a sequence of length n sits at position n - chunk + i and
+    attends to n - chunk + i + 1 keys (none if that is not positive)."""
+    keys = 0
+    for n in lens:
+        n = int(n)
+        first = n - chunk + 1  # keys of the chunk's first query
+        if first >= 1:
+            keys += chunk * (first - 1) + chunk * (chunk + 1) // 2
+        else:  # queries before the sequence start attend to nothing
+            m = max(0, n)
+            keys += m * (m + 1) // 2
+    return 4 * D * Hq * keys
+
+
 class DecodeScenario:
     def __init__(self, w: wl.Workload, fmt: str | None = None, device: str = "cuda",
                  seq_offset: int = 0, lens=None):
@@ -169,9 +186,5 @@ class DecodeScenario:
 
     @property
     def prefill_flops(self) -> int:
-        """Algorithmic FLOPs of the chunk prefill: 2 D (QK) + 2 D (PV) per
-        (query row, attended key); query i of a chunk of T at the end of a
-        sequence of length n attends to n - T + i + 1 keys."""
-        T, D, Hq = self.chunk, self.D, self.Hq
-        keys = sum(T * (int(n) - T) + T * (T + 1) // 2 for n in self.lens)
-        return 4 * D * Hq * keys
+        """Algorithmic FLOPs of the chunk prefill (see prefill_flops)."""
+        return prefill_flops(self.lens, self.chunk, self.Hq, self.D)
