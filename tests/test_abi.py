@@ -96,3 +96,33 @@ def test_prefill_argument_checks_run_on_the_host(L):
     assert call(bt=None) == 1
     assert call(ks=None) == 1               # quantized formats need both scales
     assert call(fmt=2) == 1                 # cache format differs from fmt
+
+
+def test_header_is_plain_c99_and_links(L, tmp_path):
+    """include/kvq.h compiles as C99 with warnings as errors (no CUDA or C++
+    headers needed) and a C program links against libkvq.so and calls its
+    host functions."""
+    import shutil
+    import subprocess
+
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "abi.c"
+    src.write_text(
+        '#include <stdio.h>\n#include "kvq.h"\n'
+        "int main(void) {\n"
+        "  float s = 0.f; int64_t n = 0;\n"
+        "  kvq_status a = kv_scale_from_absmax(KVQ_FMT_FP8_E4M3, 448.0f, &s);\n"
+        "  kvq_status b = kv_cache_bytes(KVQ_FMT_NVFP4, 37, 3, 128, &n);\n"
+        '  printf("%d %a %d %lld\\n", (int)a, (double)s, (int)b, (long long)n);\n'
+        "  return 0;\n}\n")
+    exe = tmp_path / "abi"
+    libdir = os.path.dirname(kbuild.LIB)
+    subprocess.run([gcc, "-std=c99", "-Wall", "-Wextra", "-Werror", "-I",
+                    os.path.join(ROOT, "include"), str(src), "-L", libdir, "-lkvq",
+                    f"-Wl,-rpath,{libdir}", "-o", str(exe)], check=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split()
+    assert out[0] == "0" and out[2] == "0"
+    assert float.fromhex(out[1]) == float(np.float32(oracle.fp8_scale(448.0)))
+    assert int(out[3]) == 37 * 3 * oracle.head_page_bytes("nvfp4", 128)
