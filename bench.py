@@ -3,23 +3,25 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl kvq|reference]
 
-One step = quantize-on-write of the step's new token per sequence (through the
-block table) + the fused-dequant decode attention over the whole context, on
-the workload "fp8-paged-4x32k": 4 sequences x 32,768 tokens, 8 KV heads, 64
-query heads, head_dim 128, FP8 E4M3 cache in 16-token pages at a random
-permutation of the pool, per-layer scales calibrated on a 16,384-token sample.
-value = KV-scan bytes per step / device time per step (GB/s).  L2 is flushed
-before every timed step (a 512 MiB write, then a 256 MiB read so no dirty
-lines are left for the timed kernel to write back).
+One step, on the workload "agents-fp8-4x127k" (4 sequences x 126,976 tokens,
+8 KV heads, 64 query heads, head_dim 128, FP8 E4M3 cache in 16-token pages at
+a random permutation of the pool, per-layer scales calibrated on a
+16,384-token sample): quantize-on-write of a 2,048-token chunk per sequence
+through the block table, then the fused-dequant decode attention over the
+whole context.  value = KV-scan bytes per step / device time per step (GB/s).
+L2 is flushed before every timed step (a 512 MiB write, then a 256 MiB read
+so no dirty lines are left for the timed kernel to write back).
 
-Extra keys report the other rows: the BF16 vs FP8 vs NVFP4 comparison on the
-1 x 65,536-token, D 64 workload, the 4 x 126,976-token agent step (2,048-token
-prefill chunk written per sequence, then decode), and the calibration abs-max.
+Extra keys (compact rows of µs, GB/s and fraction of the HBM peak) report the
+other rows: BF16 vs FP8 vs NVFP4 decode on the same 4 x 126,976-token cache
+and on the 1 x 65,536-token D=64 workload, the FP8 4 x 32,768-token paged
+step, a 4,096-token sliding window, the calibration abs-max and the chunked
+prefill of the agent step.
 
 Under torchrun (N > 1) every rank runs its own batch of sequences (weak
 scaling, no data-path collective); time is the max over ranks.
-``--impl reference`` times the CPU oracle instead (rank 0 only), on bounded
-samples of the same workload.
+``--impl reference`` times the CPU oracle instead (rank 0 only), on all host
+cores, over bounded samples of the same workload.
 """
 from __future__ import annotations
 
@@ -37,7 +39,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "decode-attn KV-scan GB/s (frac of HBM peak) & µs/step, BF16 vs FP8 vs NVFP4"
-MAIN_WORKLOAD = "fp8-paged-4x32k"
+MAIN_WORKLOAD = "agents-fp8-4x127k"
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 FALLBACK_BF16_TFLOPS_SUSTAINED = 1400.0
@@ -52,7 +54,7 @@ def parse():
     ap.add_argument("--impl", default="kvq", choices=["kvq", "reference"])
     ap.add_argument("--workload", default=MAIN_WORKLOAD)
     ap.add_argument("--no-extras", action="store_true", help="main line only")
-    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--cpu-seconds", type=float, default=6.0)
     ap.add_argument("--sweep", action="store_true",
                     help="instead of the bench line: decode time of every sweep cell "
                          "(context x batch x head_dim x format), one JSON line each")
@@ -213,67 +215,124 @@ class Timer:
         return part_ms, step_ms
 
 
-def cpu_baseline_sample(w, fmt, seconds, steps=None):
-    """The CPU oracle on bounded samples of the workload: one (sequence, KV
-    head) unit at a time, quantize-on-write of its step token(s) + float64
-    decode attention of its G query heads over the full context.  Inputs are
-    host-drawn with the same recipe.  Returns (GB/s, units, seconds)."""
-    import numpy as np
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
 
-    import oracle
-    from quantized_kv_cache_21_b200 import workloads as wl
-    from quantized_kv_cache_21_b200.scenario import kv_scan_bytes
 
-    G, D, L = w.Hq // w.Hkv, w.D, w.seq_len
-    chunk = max(1, w.write_chunk)
-    mb = -(-L // 16)
-    bt = np.arange(mb, dtype=np.int32)[None, :]
-    unit_bytes = kv_scan_bytes(fmt, [L], 1, D)
-    done, t_total, u = 0, 0.0, 0
-    while True:
+class OracleUnits:
+    """(sequence, KV head) units of a workload for the CPU oracle, each with
+    its cache already holding the context before the step's chunk.  One
+    "round" runs, for every unit, the step the GPU times: quantize-on-write
+    of the step's chunk of tokens + float64 decode attention of the KV head's
+    G query heads over the whole context.  Units are independent, so a round
+    runs them on a pool of host threads (the oracle's C calls release the
+    GIL); inputs are host-drawn with the workloads' recipe."""
+
+    def __init__(self, w, fmt, n_units, threads, first_unit=0):
+        from concurrent.futures import ThreadPoolExecutor
+
+        self.w, self.fmt, self.threads = w, fmt, threads
+        self.G, self.D, self.L = w.Hq // w.Hkv, w.D, w.seq_len
+        self.chunk = max(1, w.write_chunk)
+        self.mb = -(-self.L // 16)
+        self.pool = ThreadPoolExecutor(max_workers=threads)
+        self.units = list(self.pool.map(self._prepare, range(first_unit, first_unit + n_units)))
+
+    def _prepare(self, u):
+        import numpy as np
+
+        import oracle
+        from quantized_kv_cache_21_b200 import workloads as wl
+
+        w, L, D, G, chunk = self.w, self.L, self.D, self.G, self.chunk
         rng = wl.rng_for(w.seed, 5000 + u)
-        k = wl.make_tokens(rng, L, 1, D, [(0, 3)] if w.outlier_factor != 1 else [],
-                           w.outlier_factor)
-        v = wl.make_tokens(rng, L, 1, D)
+        outl = [(0, 3)] if w.outlier_factor != 1 else []
+        k = wl.make_tokens(rng, L, 1, D, outl, w.outlier_factor)
+        v = wl.make_tokens(rng, L, 1, D, outl, w.outlier_factor)
         q = wl.make_query(rng, 1, G, D)
         n = L if w.calib_tokens is None else w.calib_tokens
-        ks = oracle.scale_from_absmax(fmt, oracle.absmax_bf16(k[:n]))
-        vs = oracle.scale_from_absmax(fmt, oracle.absmax_bf16(v[:n]))
-        kc, vc = oracle.new_cache(fmt, mb, 1, D)
+        ks = oracle.scale_from_absmax(self.fmt, oracle.absmax_bf16(k[:n]))
+        vs = oracle.scale_from_absmax(self.fmt, oracle.absmax_bf16(v[:n]))
+        kc, vc = oracle.new_cache(self.fmt, self.mb, 1, D)
         slots = np.arange(L, dtype=np.int64)
-        oracle.write(fmt, k[: L - chunk], v[: L - chunk], slots[: L - chunk], kc, vc, ks, vs)
+        oracle.write(self.fmt, k[: L - chunk], v[: L - chunk], slots[: L - chunk], kc, vc, ks, vs)
+        return dict(k=k[L - chunk:].copy(), v=v[L - chunk:].copy(), slots=slots[L - chunk:].copy(),
+                    q=q, kc=kc, vc=vc, ks=ks, vs=vs, bt=np.arange(self.mb, dtype=np.int32)[None],
+                    lens=np.array([L], np.int32))
+
+    def _step(self, x):
+        import oracle
+        oracle.write(self.fmt, x["k"], x["v"], x["slots"], x["kc"], x["vc"], x["ks"], x["vs"])
+        oracle.decode_attention(self.fmt, x["q"], x["kc"], x["vc"], 1, x["bt"], x["lens"],
+                                x["ks"], x["vs"])
+
+    def round(self) -> float:
+        """Wall seconds of one round over all units."""
         t0 = time.perf_counter()
-        oracle.write(fmt, k[L - chunk:], v[L - chunk:], slots[L - chunk:], kc, vc, ks, vs)
-        oracle.decode_attention(fmt, q, kc, vc, 1, bt, np.array([L], np.int32), ks, vs)
-        t_total += time.perf_counter() - t0
-        done += 1
-        u += 1
-        if (steps is not None and done >= steps) or (steps is None and t_total >= seconds):
-            break
-    return done * unit_bytes / t_total / 1e9, done, t_total, unit_bytes
+        list(self.pool.map(self._step, self.units))
+        return time.perf_counter() - t0
+
+    @property
+    def unit_bytes(self) -> int:
+        from quantized_kv_cache_21_b200.scenario import kv_scan_bytes
+        return kv_scan_bytes(self.fmt, [self.L], 1, self.D)
+
+    def describe(self, rounds: int, secs: float) -> str:
+        return (f"{rounds} round(s) of {len(self.units)} (sequence, KV head) unit(s) of "
+                f"{self.w.name} on {self.threads} thread(s), {secs:.1f} s; a unit = write of "
+                f"{self.chunk} token(s) + float64 attention of {self.G} heads over {self.L} "
+                f"tokens ({self.unit_bytes} KV bytes)")
+
+    def close(self):
+        self.pool.shutdown()
+
+
+def cpu_baseline(w, fmt, seconds):
+    """The oracle on all host cores (one unit per thread, rounds for about
+    `seconds`), then on one core (the first unit's step alone, once)."""
+    threads = min(host_cores(), 64)
+    ou = OracleUnits(w, fmt, threads, threads)
+    rounds, secs = 0, 0.0
+    while secs < seconds or rounds == 0:
+        secs += ou.round()
+        rounds += 1
+    allc = (rounds * len(ou.units) * ou.unit_bytes / secs / 1e9, threads,
+            ou.describe(rounds, secs))
+    t0 = time.perf_counter()
+    ou._step(ou.units[0])
+    one = ou.unit_bytes / (time.perf_counter() - t0) / 1e9
+    ou.close()
+    return {"all": allc, "one": (one, 1, "")}
 
 
 def run_reference(args):
-    """--impl reference: the CPU oracle on this workload (rank 0 only)."""
+    """--impl reference: the CPU oracle on this workload (rank 0 only), on all
+    host cores: one step = one round over one (sequence, KV head) unit per
+    thread."""
     world, rank, _ = dist_env()
     if rank != 0:
         return 0
     from quantized_kv_cache_21_b200 import workloads as wl
     w = wl.WORKLOADS[args.workload]
-    cpu_baseline_sample(w, w.fmt, 0, steps=max(1, args.warmup))  # warm-up units
-    gbps, units, secs, unit_bytes = cpu_baseline_sample(w, w.fmt, 0, steps=args.steps)
-    ms = secs / units * 1e3
-    sample = (f"{units} (sequence, KV head) units of {args.workload}, each: quantize-on-write "
-              f"of {max(1, w.write_chunk)} token(s) + float64 decode attention of "
-              f"{w.Hq // w.Hkv} query heads over {w.seq_len} tokens ({unit_bytes} KV bytes)")
+    threads = min(host_cores(), 64)
+    ou = OracleUnits(w, w.fmt, threads, threads)
+    for _ in range(args.warmup):
+        ou.round()
+    times = [ou.round() for _ in range(args.steps)]
+    secs = sum(times)
+    gbps = args.steps * threads * ou.unit_bytes / secs / 1e9
     line = {"impl": "reference", "metric": METRIC, "value": gbps, "unit": "GB/s",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "f64", "data": "synthetic", "config": workload_config(w),
-            "cpu_baseline": {"value": gbps, "unit": "GB/s", "cores": 1, "kind": "oracle",
-                             "sample": sample},
+            "ms_per_step": secs / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": workload_config(w),
+            "cpu_baseline": {"value": gbps, "unit": "GB/s", "cores": threads, "kind": "oracle",
+                             "sample": ou.describe(args.steps, secs)},
             "e2e": {"value": gbps, "unit": "GB/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
+    ou.close()
     print(json.dumps(line))
     return 0
 
@@ -344,6 +403,18 @@ def run_sweep(args):
     return 0
 
 
+def r4(x):
+    """Four significant digits (keeps the JSON line short)."""
+    return float(f"{x:.4g}") if x is not None else None
+
+
+def row(bytes_, ms_list, peak):
+    """Compact timing row of a decode-like launch: µs, GB/s, fraction of peak."""
+    ms = statistics.mean(ms_list)
+    gbps = bytes_ / (ms * 1e-3) / 1e9
+    return {"us": r4(ms * 1e3), "GBps": r4(gbps), "frac": r4(gbps / peak)}
+
+
 def main():
     args = parse()
     if args.impl == "reference":
@@ -370,14 +441,16 @@ def main():
     peak, peak_kind = measured_hbm_peak()
     K, W = args.steps, max(3, args.warmup)
 
-    # ---------------- main line: write + decode step
+    # ---------------- main line: quantize-on-write of the step's tokens, then
+    # the fused-dequant decode over the whole context, timed as one part (no
+    # event between the two launches: the decode's prologue may overlap the
+    # write's tail, as in a serving loop)
     w = wl.WORKLOADS[args.workload]
     sc = DecodeScenario(w, device="cuda", seq_offset=rank * w.B)
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
-    # The step (write, then decode) is timed as one part: no event between the
-    # two launches, so the decode may start its prologue while the write ends.
+
     def step():
         sc.write()
         sc.decode()
@@ -390,8 +463,8 @@ def main():
     max_total_ms = reduce_max(total_ms, world, device="cuda")
 
     # ---------------- end to end through the public API with host buffers:
-    # one pinned upload of the step's inputs (q, step K, step V) and one pinned
-    # download of its results (out, lse) per step, around the write + decode
+    # one pinned upload of the step's inputs (q, the step's K and V tokens)
+    # and one pinned download of its results (out, lse) per step
     nq, nk = sc.q.numel(), sc.step_k.numel()
     up_h = torch.empty(nq + 2 * nk, dtype=torch.bfloat16).pin_memory()
     up_h[:nq].copy_(sc.q.reshape(-1).cpu())
@@ -414,28 +487,11 @@ def main():
 
     if world > 1:
         torch.distributed.barrier()
-    _, e2e_eager_ms = timer.run([e2e_step], K, W)
-    # The same step captured once in a CUDA graph (the same API calls; the
-    # write -> decode programmatic dependency is kept as a graph edge) and
-    # replayed: what a serving loop does to drop per-call launch overhead.
-    torch.cuda.synchronize()
-    side = torch.cuda.Stream()
-    side.wait_stream(torch.cuda.current_stream())
-    with torch.cuda.stream(side):
-        for _ in range(2):
-            e2e_step()
-    torch.cuda.current_stream().wait_stream(side)
-    torch.cuda.synchronize()
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph):
-        e2e_step()
-    torch.cuda.synchronize()
-    _, e2e_ms = timer.run([graph.replay], K, W)
+    _, e2e_ms = timer.run([e2e_step], K, W)
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
     max_e2e_ms = reduce_max(sum(e2e_ms), world, device="cuda") / K
-    max_e2e_eager_ms = reduce_max(sum(e2e_eager_ms), world, device="cuda") / K
     assert int(sc.err.item()) == 0, f"device error word {int(sc.err.item())}"
     if rank != 0:
         if world > 1:
@@ -445,148 +501,98 @@ def main():
     ms_per_step = max_total_ms / K
     value = world * sc.scan_bytes / (ms_per_step * 1e-3) / 1e9
     line = {"metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": K,
-            "warmup": W, "ms_per_step": ms_per_step, "us_per_step": ms_per_step * 1e3,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "fp8_e4m3 (f16 mma, fp32 accumulate)",
-            "data": "synthetic: seeded N(0,1) K/V/Q in BF16, 1% outlier channels x16, "
+            "warmup": W, "ms_per_step": ms_per_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None,
+            "dtype": f"{w.fmt} cache (f16 mma, fp32 accumulate)",
+            "data": "synthetic: seeded N(0,1) BF16 K/V/Q, 1% outlier channels x16, "
                     "random block table",
             "config": dict(workload_config(w), parallelism=f"dp{world} (sequences per rank)",
                            kv_scan_bytes_per_step=sc.scan_bytes,
                            write_tokens_per_step=int(sc.step_k.shape[0]))}
-    line["frac_of_hbm_peak"] = value / world / peak
-    # each launch alone (after an L2 flush) for the roofline and the breakdown
+    # the decode launched alone after a flush: the dominant kernel's roofline
     (decode_ms,), _ = timer.run([sc.decode], K, W)
     (write_ms,), _ = timer.run([sc.write], K, W)
     line["roofline"] = roofline(sc.scan_bytes, decode_ms, peak, peak_kind,
                                 profiled_traffic(w.name))
-    line["step_breakdown_us"] = {"write_alone": statistics.mean(write_ms) * 1e3,
-                                 "decode_alone": statistics.mean(decode_ms) * 1e3,
-                                 "step": ms_per_step * 1e3}
+    line["e2e"] = {"value": world * sc.scan_bytes / (max_e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+                   "h2d_bytes_per_step": up_h.numel() * 2,
+                   "d2h_bytes_per_step": down_h.numel() * 4,
+                   "us_per_step": r4(max_e2e_ms * 1e3)}
     line["gpu_launches"] = 2 * K
-    line["e2e"] = {"value": world * sc.scan_bytes / (max_e2e_eager_ms * 1e-3) / 1e9,
-                   "unit": "GB/s", "h2d_bytes_per_step": up_h.numel() * 2,
-                   "d2h_bytes_per_step": down_h.numel() * 4, "us_per_step": max_e2e_eager_ms * 1e3,
-                   "copies_per_step": {"h2d": 1, "d2h": 1},
-                   "launch": "the API called from Python every step"}
-    line["e2e_graph"] = {"value": world * sc.scan_bytes / (max_e2e_ms * 1e-3) / 1e9,
-                         "unit": "GB/s", "us_per_step": max_e2e_ms * 1e3,
-                         "launch": "CUDA graph of the same calls, replayed each step"}
-
+    line["step_us"] = {"step": r4(ms_per_step * 1e3), "write": r4(statistics.mean(write_ms) * 1e3),
+                       "decode": r4(statistics.mean(decode_ms) * 1e3)}
     del sc
     torch.cuda.empty_cache()
 
-    # ---------------- other rows
+    extras = {}
     if not args.no_extras:
-        wf = wl.WORKLOADS["nvfp4-1x64k"]
-        fm = {}
-        for fmt in ("bf16", "fp8", "nvfp4"):
-            s2 = DecodeScenario(wf, fmt=fmt, device="cuda")
-            (dms,), _ = timer.run([s2.decode], K, W)
-            a = s2.scan_bytes / (statistics.mean(dms) * 1e-3) / 1e9
-            fm[fmt] = {"us_per_step": statistics.mean(dms) * 1e3, "kv_scan_bytes": s2.scan_bytes,
-                       "GBps": a, "frac_of_hbm_peak": a / peak}
-            assert int(s2.err.item()) == 0
-            del s2
-            torch.cuda.empty_cache()
-        fm["config"] = workload_config(wf, "bf16|fp8|nvfp4")
-        fm["speedup_vs_bf16"] = {f: fm["bf16"]["us_per_step"] / fm[f]["us_per_step"]
-                                 for f in ("fp8", "nvfp4")}
-        line["formats"] = fm
-
+        Kx = max(3, K // 2)
+        # chunked prefill of the agent step: each sequence's 2,048-token chunk
+        # attends causally to its 126,976 cached tokens (tensor-core bound)
         wa = wl.WORKLOADS["agents-fp8-4x127k"]
         s3 = DecodeScenario(wa, device="cuda")
-        Ka = max(3, K // 4)
-
-        def step3():
-            s3.write()
-            s3.decode()
-
-        _, sms = timer.run([step3], Ka, W)
-        (wms,), _ = timer.run([s3.write], Ka, W)
-        (dms,), _ = timer.run([s3.decode], Ka, W)
-        line["agents"] = {"config": dict(workload_config(wa),
-                                         write_tokens_per_step=int(s3.step_k.shape[0])),
-                          "us_per_step": statistics.mean(sms) * 1e3,
-                          "write_alone_us": statistics.mean(wms) * 1e3,
-                          "decode_alone_us": statistics.mean(dms) * 1e3,
-                          "decode_GBps": s3.scan_bytes / (statistics.mean(dms) * 1e-3) / 1e9,
-                          "decode_frac_of_hbm_peak":
-                              s3.scan_bytes / (statistics.mean(dms) * 1e-3) / 1e9 / peak}
-        assert int(s3.err.item()) == 0
-
-        # chunked prefill on the same cache: each sequence's 2,048-token chunk
-        # (written above) attends causally to its 126,976 cached tokens;
-        # tensor-core bound, so reported against the bf16 dense peak
         s3.prefill_setup()
         s3.write()
         (pms,), _ = timer.run([s3.prefill], 3, W)
         assert int(s3.err.item()) == 0
-        t_pf = statistics.mean(pms) * 1e-3
         pk_s, pk_b, pk_kind = measured_tensor_peak()
-        tf = s3.prefill_flops / t_pf / 1e12
-        line["chunked_prefill"] = {
-            "config": dict(workload_config(wa), chunk_tokens_per_seq=s3.chunk,
-                           attention="causal: query i of the chunk sees positions <= its own"),
-            "ms_per_launch": t_pf * 1e3, "algorithmic_flops": s3.prefill_flops,
-            "TFLOPs": tf, "peak_TFLOPs": pk_s, "peak": f"{pk_kind} bf16 dense, sustained",
-            "frac_of_tensor_peak": tf / pk_s, "frac_of_burst_peak": tf / pk_b,
-            "mma": "tcgen05.mma kind::f16 (bf16 for BF16 pages), M=128, fp32 accumulators in "
-                   "tensor memory; P enters PV as two 16-bit halves (executed MMA flops = 1.5x "
-                   "algorithmic)"}
+        tf = s3.prefill_flops / (statistics.mean(pms) * 1e-3) / 1e12
+        extras["chunked_prefill_4x127k"] = {
+            "ms": r4(statistics.mean(pms)), "TFLOPs": r4(tf),
+            "frac_sustained": r4(tf / pk_s), "peak_TFLOPs": pk_s, "peak": pk_kind}
         del s3
         torch.cuda.empty_cache()
 
-        # the same 4 x 126,976-token, head_dim-128 cache in all three formats:
-        # the byte-heavy comparison (decode launches only)
-        af = {}
-        for fmt in ("bf16", "fp8", "nvfp4"):
-            s4 = DecodeScenario(wa, fmt=fmt, device="cuda")
-            (dms,), _ = timer.run([s4.decode], max(3, K // 4), W)
-            a = s4.scan_bytes / (statistics.mean(dms) * 1e-3) / 1e9
-            af[fmt] = {"us_per_step": statistics.mean(dms) * 1e3, "kv_scan_bytes": s4.scan_bytes,
-                       "GBps": a, "frac_of_hbm_peak": a / peak}
-            assert int(s4.err.item()) == 0
-            del s4
-            torch.cuda.empty_cache()
-        af["config"] = workload_config(wa, "bf16|fp8|nvfp4")
-        af["speedup_vs_bf16"] = {f: af["bf16"]["us_per_step"] / af[f]["us_per_step"]
-                                 for f in ("fp8", "nvfp4")}
-        line["agents_formats"] = af
-
-        # sliding-window mode ("SWA mode" of the MI300X benchmark page: window
-        # 4096) on the main workload's cache: decode launches only
-        s5 = DecodeScenario(w, device="cuda")
-        swa = {}
-        for win in (4096,):
-            s5.window_ws(win)
-            (dms,), _ = timer.run([lambda: s5.decode_window(win)], K, W)
-            b5 = s5.window_scan_bytes(win)
-            a = b5 / (statistics.mean(dms) * 1e-3) / 1e9
-            swa[str(win)] = {"us_per_step": statistics.mean(dms) * 1e3, "kv_scan_bytes": b5,
-                             "GBps": a, "frac_of_hbm_peak": a / peak}
-        assert int(s5.err.item()) == 0
-        line["sliding_window"] = {"config": dict(workload_config(w), window="last 4096 tokens"),
-                                  "windows": swa}
-        del s5
-        torch.cuda.empty_cache()
-
+        # the calibration abs-max over 65,536 x 8 x 128 BF16
         x = wl.device_tokens(20264, 0, 65536, 8, 128)
         amax = torch.zeros(1, dtype=torch.float32, device="cuda")
         (cms,), _ = timer.run([lambda: kvq.kv_calibrate_absmax(x, amax)], K, W)
-        cb = x.numel() * 2
-        line["calibration"] = {"tensor": "65,536 x 8 x 128 BF16", "bytes": cb,
-                               "us": statistics.mean(cms) * 1e3,
-                               "GBps": cb / (statistics.mean(cms) * 1e-3) / 1e9}
+        extras["calibration_64k"] = row(x.numel() * 2, cms, peak)
         del x
 
+        # the FP8 4 x 32,768-token paged workload: the step (4-token write +
+        # decode), the decode alone, and a sliding window of 4,096 tokens
+        wp = wl.WORKLOADS["fp8-paged-4x32k"]
+        s1 = DecodeScenario(wp, device="cuda")
+
+        def step1():
+            s1.write()
+            s1.decode()
+
+        (s1ms,), _ = timer.run([step1], K, W)
+        (d1ms,), _ = timer.run([s1.decode], K, W)
+        s1.window_ws(4096)
+        (w1ms,), _ = timer.run([lambda: s1.decode_window(4096)], K, W)
+        assert int(s1.err.item()) == 0
+        extras["swa4096_4x32k"] = row(s1.window_scan_bytes(4096), w1ms, peak)
+        extras["paged_4x32k"] = {"step": row(s1.scan_bytes, s1ms, peak),
+                                 "decode": row(s1.scan_bytes, d1ms, peak)}
+        del s1
+        torch.cuda.empty_cache()
+
+        # BF16 vs FP8 vs NVFP4 decode on the byte-heavy 4 x 126,976-token
+        # D=128 cache and on the 1 x 65,536-token D=64 workload
+        for key, name, reps in (("formats_4x127k", "agents-fp8-4x127k", Kx),
+                                ("formats_1x64k", "nvfp4-1x64k", K)):
+            wf = wl.WORKLOADS[name]
+            fm = {}
+            for fmt in ("bf16", "fp8", "nvfp4"):
+                s2 = DecodeScenario(wf, fmt=fmt, device="cuda")
+                (dms,), _ = timer.run([s2.decode], reps, W)
+                assert int(s2.err.item()) == 0
+                fm[fmt] = row(s2.scan_bytes, dms, peak)
+                del s2
+                torch.cuda.empty_cache()
+            extras[key] = fm
+
     line["clocks"] = clocks.summary()
-    if world == 1:
-        gbps, units, secs, unit_bytes = cpu_baseline_sample(w, w.fmt, args.cpu_seconds)
-        line["cpu_baseline"] = {
-            "value": gbps, "unit": "GB/s", "cores": 1, "kind": "oracle",
-            "sample": f"{units} (sequence, KV head) units of {w.name} ({unit_bytes} KV bytes "
-                      f"each: write of the step token + float64 attention of "
-                      f"{w.Hq // w.Hkv} heads over {w.seq_len} tokens), {secs:.1f} s"}
+    if world == 1 and args.cpu_seconds > 0:
+        cb = cpu_baseline(w, w.fmt, args.cpu_seconds)
+        gbps, cores, sample = cb["all"]
+        line["cpu_baseline"] = {"value": gbps, "unit": "GB/s", "cores": cores, "kind": "oracle",
+                                "sample": sample, "one_core_GBps": r4(cb["one"][0])}
+    line["peak_GBps"] = {"value": peak, "source": peak_kind}
+    line.update(extras)
     print(json.dumps(line))
     if world > 1:
         torch.distributed.barrier()

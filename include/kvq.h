@@ -19,8 +19,14 @@
  *
  * Conventions shared by every entry point
  *   - All tensor pointers are DEVICE pointers owned by the caller.  The
- *     library allocates no device memory and keeps no state except a
- *     per-device capability check.
+ *     library allocates no device memory at run time.  The host state it
+ *     keeps is small and safe to share between threads: per device ordinal,
+ *     the capability check, the SM count and whether each kernel's shared-
+ *     memory limit has been raised; per calling thread, the text of the last
+ *     error and the TMA descriptors of the last few caches it decoded (keyed
+ *     by device, buffer addresses and geometry, so a reused address with the
+ *     same geometry encodes the same descriptor).  The only device state is
+ *     the fixed scratch array of kv_decode_attention_static_ws (below).
  *   - Every call is asynchronous on the given stream (a cudaStream_t passed
  *     as kvq_stream; NULL means the legacy default stream) and never
  *     synchronises.

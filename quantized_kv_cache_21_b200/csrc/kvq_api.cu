@@ -242,6 +242,18 @@ kvq_status cached_maps(int fmt, const kvq_cache* c, const CUtensorMap** out) {
 namespace kvq {
 void set_last_error(const char* msg) { snprintf(g_err, sizeof(g_err), "%s", msg); }
 
+cudaError_t ensure_smem_attr(const void* func, size_t bytes, std::atomic<bool>* done) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const bool tracked = dev >= 0 && dev < kMaxDevices;
+  if (tracked && done[dev].load(std::memory_order_acquire)) return cudaSuccess;
+  e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(bytes));
+  if (e == cudaSuccess && tracked) done[dev].store(true, std::memory_order_release);
+  return e;
+}
+
 int num_sms() {
   static std::atomic<int> cached[64];  // per device ordinal; 0 = not yet asked
   int dev = 0, n = 0;

@@ -762,6 +762,15 @@ __global__ void __launch_bounds__(Shape<FMT, D>::NW * 32, 1)
     if (!scale_ok && c == 0 && tid == 0) set_err(p.d_err, kErrScale);
   }
 
+  // Scores are scaled by c = sm_scale * k_scale * log2(e) in the softmax
+  // below, and masked tokens carry a raw score of -inf, so c must be positive:
+  // a negative sm_scale is moved into Q's sign (exact), and c = 0 (an all-zero
+  // NVFP4 K tensor, g = 0, whose scores are all 0) becomes a tiny positive c
+  // with the same result.
+  const float c_raw = p.sm_scale * ks * kLog2e;
+  const uint32_t q_sign = c_raw < 0.f ? 0x80008000u : 0u;
+  const float c_log2 = fmaxf(fabsf(c_raw), 1e-30f);
+
   // Query fragments (B operand of QK) of unit u; padded heads are 0.  The
   // thread's head-dim elements come in 16-byte runs of 8.
   uint32_t qb[KS][2];
@@ -779,7 +788,7 @@ __global__ void __launch_bounds__(Shape<FMT, D>::NW * 32, 1)
       for (int x = 0; x < 4; ++x) {
         uint32_t v = ws[x];
         if constexpr (!F::kBF16) v = pack_f16x2(bf16_lo(v), bf16_hi(v));
-        qb[i / 4 + x / 2][x & 1] = v;
+        qb[i / 4 + x / 2][x & 1] = v ^ q_sign;
       }
     }
   };
@@ -911,7 +920,6 @@ __global__ void __launch_bounds__(Shape<FMT, D>::NW * 32, 1)
     }
   }
 
-  const float c_log2 = p.sm_scale * ks * kLog2e;
   int k_base = 0, j = 0;  // j = this warp's next local item
   int st = 0, ph = 0;     // its stage (j % NSW) and barrier phase parity ((j / NSW) & 1)
   for (int si = 0; si < nu; ++si) {
@@ -1183,14 +1191,10 @@ cudaError_t launch_t(const CUtensorMap* maps, const DecodeParams& p, int ctas,
                      cudaStream_t stream) {
   using S = Shape<FMT, D>;
   const size_t smem = smem_bytes<FMT, D>();
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(kvq_decode_kernel<FMT, D>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static std::atomic<bool> attr_done[kMaxDevices];  // per device ordinal
+  cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kvq_decode_kernel<FMT, D>),
+                                   smem, attr_done);
+  if (e != cudaSuccess) return e;
   // Programmatic stream serialization: the launch may begin while a
   // preceding kv_quantize_write of this stream finishes (see griddep_wait).
   cudaLaunchConfig_t cfg = {};

@@ -7,6 +7,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <atomic>
+
 namespace kvq {
 
 struct DecodeParams {
@@ -94,6 +96,14 @@ cudaError_t launch_absmax(const uint16_t* x, int64_t n, float* d_amax, cudaStrea
 cudaError_t launch_scale(int fmt, const float* d_amax, float* d_scale, cudaStream_t stream);
 
 int num_sms();
+
+// Raises a kernel's dynamic shared-memory limit to `bytes` on the current
+// device, once per device: `done` is the kernel's own per-device-ordinal flag
+// array (kMaxDevices entries, zero-initialised).  The attribute belongs to the
+// device's context, so a kernel launched on a second GPU sets it there again;
+// concurrent first calls may both set it, which is harmless.
+constexpr int kMaxDevices = 64;
+cudaError_t ensure_smem_attr(const void* func, size_t bytes, std::atomic<bool>* done);
 // Sets the text kvq_last_error() returns on this thread.
 void set_last_error(const char* msg);
 

@@ -527,15 +527,11 @@ __global__ void __launch_bounds__(kThreads, 2) kvq_prefill_kernel(const PrefillP
 
 template <int FMT, int D>
 cudaError_t launch_t(const PrefillParams& p, int64_t ctas, cudaStream_t stream) {
-  static bool attr_set = false;  // per instantiation; the attribute is per function
+  static std::atomic<bool> attr_done[kMaxDevices];  // per instantiation and device ordinal
   constexpr size_t smem = smem_bytes<D>();
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(kvq_prefill_kernel<FMT, D>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kvq_prefill_kernel<FMT, D>),
+                                   smem, attr_done);
+  if (e != cudaSuccess) return e;
   kvq_prefill_kernel<FMT, D><<<static_cast<unsigned>(ctas), kThreads, smem, stream>>>(p);
   return cudaGetLastError();
 }

@@ -37,7 +37,9 @@ class Case:
     library) and an oracle cache (by the oracle), plus the query."""
 
     def __init__(self, fmt, B, Hkv, Hq, D, lens, seed, permuted=True, factor=8.0,
-                 outliers_per_head=1, extra_blocks=3, fill=0, calib_tokens=None):
+                 outliers_per_head=1, extra_blocks=3, fill=0, calib_tokens=None, zero_k=False):
+        """zero_k: K is all zeros (its abs-max is 0, so the NVFP4 global scale
+        g is 0 and every score is 0)."""
         rng = wl.rng_for(seed, 0)
         self.fmt, self.B, self.Hkv, self.Hq, self.D = fmt, B, Hkv, Hq, D
         self.lens = np.array(lens, np.int32)
@@ -50,6 +52,8 @@ class Case:
             self.bt = wl.identity_block_table(B, self.max_blocks)
         outl = wl.outlier_pairs(rng, Hkv, D, per_head=outliers_per_head) if factor != 1 else []
         self.k = [wl.make_tokens(rng, int(n), Hkv, D, outl, factor) for n in self.lens]
+        if zero_k:
+            self.k = [np.zeros_like(k) for k in self.k]
         self.v = [wl.make_tokens(rng, int(n), Hkv, D, outl, factor) for n in self.lens]
         self.q = wl.make_query(rng, B, Hq, D)
         kc = np.concatenate(self.k) if self.k else np.zeros((0, Hkv, D), np.uint16)

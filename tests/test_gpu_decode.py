@@ -6,6 +6,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 import quantized_kv_cache_21_b200 as kvq
 from quantized_kv_cache_21_b200 import workloads as wl
 
@@ -114,6 +115,58 @@ def test_custom_sm_scale():
     c = Case("fp8", 1, 2, 8, 64, [200], seed=4600)
     out, lse = c.decode(sm_scale=0.05)
     assert_attention_close(out, lse, *c.reference(sm_scale=0.05))
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("splits", [0, 3])
+def test_negative_sm_scale(fmt, D, splits):
+    """A negative softmax scale is a finite sm_scale the interface accepts:
+    the scores change sign, and the masked tail of every partial last page
+    (lengths 1, 15, 17, 1001) must still carry no weight."""
+    c = Case(fmt, 4, 2, 16, D, [1, 15, 17, 1001], seed=4650 + D, factor=16.0)
+    out, lse = c.decode(num_splits=splits, sm_scale=-0.08)
+    assert int(c.err.item()) == 0
+    assert_attention_close(out, lse, *c.reference(sm_scale=-0.08))
+
+
+def mean_of_v_hat(c: Case):
+    """[B][Hq][D]: the mean over each sequence's tokens of the oracle's
+    dequantised V at the query head's KV head (the exact result when every
+    score is equal)."""
+    G = c.Hq // c.Hkv
+    out = np.zeros((c.B, c.Hq, c.D))
+    for b in range(c.B):
+        n = int(c.lens[b])
+        if n == 0:
+            continue
+        slots = wl.physical_slots(c.bt, b, np.arange(n))
+        _, v_hat = oracle.dequantize(c.fmt, c.okc, c.ovc, c.Hkv, c.D, slots, c.ks, c.vs)
+        mean = v_hat.astype(np.float64).mean(axis=0)  # [Hkv][D]
+        out[b] = np.repeat(mean, G, axis=0)
+    return out
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("splits", [0, 3])
+def test_all_zero_k(fmt, D, splits):
+    """An all-zero K tensor: its abs-max is 0, so the NVFP4 global scale g is
+    0 (the FP8 scale is the 1e-12 floor) and every score is exactly 0.  The
+    result is the plain mean of the dequantised V and lse = ln T, also on
+    lengths that end inside a page."""
+    lens = [1, 15, 17, 1001]
+    c = Case(fmt, 4, 2, 16, D, lens, seed=4660 + D, factor=16.0, zero_k=True)
+    if fmt == "nvfp4":
+        assert c.ks == 0.0
+    out, lse = c.decode(num_splits=splits)
+    assert int(c.err.item()) == 0
+    ref_out, ref_lse = c.reference()
+    assert_attention_close(out, lse, ref_out, ref_lse)
+    np.testing.assert_allclose(ref_lse, np.log(np.array(lens, np.float64))[:, None]
+                               * np.ones((1, c.Hq)), rtol=1e-12)
+    np.testing.assert_allclose(lse, ref_lse, rtol=1e-6, atol=1e-5)
+    assert np.abs(out - mean_of_v_hat(c)).max() <= 2e-3
 
 
 def test_bad_block_id_and_seq_len_are_reported():
@@ -240,3 +293,45 @@ def test_bounded_wait_times_out_and_reports():
     out, lse = c.decode()
     assert int(c.err.item()) == 0
     assert_attention_close(out, lse, *c.reference())
+
+
+def test_decode_from_two_host_threads_on_one_stream():
+    """Two host threads launch decodes of different formats and head dims on
+    one shared stream at the same time (the library's per-device launch state
+    is shared between them); every result matches the oracle."""
+    import threading
+
+    cases = [Case("fp8", 2, 2, 16, 128, [3000, 1200], seed=7800, factor=16.0),
+             Case("nvfp4", 3, 2, 16, 64, [900, 17, 2500], seed=7801, factor=16.0)]
+    stream = torch.cuda.Stream()
+    outs = []
+    for c in cases:
+        msl = c.max_blocks * 16
+        ws = kvq.new_workspace(kvq.kv_decode_workspace_size(c.fmt, c.B, c.Hq, c.Hkv, c.D, msl))
+        outs.append((torch.full((c.B, c.Hq, c.D), float("nan"), device=DEV),
+                     torch.full((c.B, c.Hq), float("nan"), device=DEV), ws, msl))
+    torch.cuda.synchronize()
+    start = threading.Barrier(2)
+    errors = []
+
+    def run(i):
+        try:
+            c = cases[i]
+            out, lse, ws, msl = outs[i]
+            start.wait()
+            for _ in range(3):
+                kvq.kv_decode_attention(c.fmt, c.d_q, c.cache, c.d_bt, c.d_lens, msl, c.d_ks,
+                                        c.d_vs, out, lse, ws, c.err, stream=stream)
+        except Exception as e:  # surfaced by the main thread
+            errors.append(e)
+
+    threads = [threading.Thread(target=run, args=(i,)) for i in range(2)]
+    for t in threads:
+        t.start()
+    for t in threads:
+        t.join()
+    assert not errors, errors
+    torch.cuda.synchronize()
+    for c, (out, lse, _, _) in zip(cases, outs):
+        assert int(c.err.item()) == 0
+        assert_attention_close(out.cpu().numpy(), lse.cpu().numpy(), *c.reference())

@@ -18,21 +18,21 @@ pytestmark = pytest.mark.gpu
 FMTS = ["bf16", "fp8", "nvfp4"]
 
 
-def decode_window(c: Case, W: int, num_splits: int = 0):
+def decode_window(c: Case, W: int, num_splits: int = 0, sm_scale: float = 0.0):
     msl = c.max_blocks * 16
     ws = kvq.new_workspace(kvq.kv_decode_workspace_size_window(c.fmt, c.B, c.Hq, c.Hkv, c.D, msl,
                                                                W, num_splits))
     out = torch.full((c.B, c.Hq, c.D), float("nan"), device=DEV)
     lse = torch.full((c.B, c.Hq), float("nan"), device=DEV)
     kvq.kv_decode_attention_window(c.fmt, c.d_q, c.cache, c.d_bt, c.d_lens, msl, W, c.d_ks,
-                                   c.d_vs, out, lse, ws, c.err, 0.0, num_splits)
+                                   c.d_vs, out, lse, ws, c.err, sm_scale, num_splits)
     torch.cuda.synchronize()
     return out.cpu().numpy(), lse.cpu().numpy()
 
 
-def reference_window(c: Case, W: int):
+def reference_window(c: Case, W: int, sm_scale=None):
     return oracle.decode_attention(c.fmt, c.q, c.okc, c.ovc, c.Hkv, c.bt, c.lens, c.ks, c.vs,
-                                   window=W)
+                                   sm_scale=sm_scale, window=W)
 
 
 @pytest.mark.parametrize("fmt", FMTS)
@@ -80,3 +80,24 @@ def test_window_zero_is_the_full_decode():
 def test_negative_window_is_rejected():
     with pytest.raises(kvq.KvqError, match="window"):
         kvq.kv_decode_workspace_size_window("fp8", 1, 8, 1, 64, 100, -1)
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("splits", [0, 2])
+def test_window_negative_scale_and_zero_k(fmt, D, splits):
+    """W = 37 starts inside a page, so the window's first page has masked
+    tokens before it: with a negative sm_scale, and with an all-zero K (NVFP4
+    g = 0, every score 0: out = mean of the window's V, lse = ln min(W, T))."""
+    lens = [1, 15, 17, 1001]
+    c = Case(fmt, 4, 2, 16, D, lens, seed=6500 + D, factor=16.0)
+    out, lse = decode_window(c, 37, splits, sm_scale=-0.08)
+    assert int(c.err.item()) == 0
+    assert_attention_close(out, lse, *reference_window(c, 37, sm_scale=-0.08))
+    z = Case(fmt, 4, 2, 16, D, lens, seed=6510 + D, factor=16.0, zero_k=True)
+    out, lse = decode_window(z, 37, splits)
+    assert int(z.err.item()) == 0
+    ref_out, ref_lse = reference_window(z, 37)
+    assert_attention_close(out, lse, ref_out, ref_lse)
+    n = np.minimum(np.array(lens, np.float64), 37)
+    np.testing.assert_allclose(lse, np.log(n)[:, None] * np.ones((1, z.Hq)), rtol=1e-6, atol=1e-5)

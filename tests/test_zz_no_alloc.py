@@ -4,9 +4,9 @@ decode step (a fixed memory pool they must not bypass, no room for a
 cudaMalloc's latency, no scratch handed to them).  It uses a fixed 8 MiB
 scratch array built into the library instead of a caller workspace.
 
-Checked through the C ABI against the regular entry point (caller
-workspace) on two calls in a row, within the attention tolerance the other
-parity tests use, and for its size limit.  This file is collected last so a
+Checked through the C ABI against the float64 CPU oracle and against the
+regular entry point (caller workspace) on two calls in a row, within the
+attention tolerance the other parity tests use, and for its size limit.  This file is collected last so a
 run that stops at the first failure has run every other test first."""
 import ctypes
 
@@ -16,7 +16,8 @@ import torch
 
 import quantized_kv_cache_21_b200 as kvq
 
-from gpu_common import DEV, LSE_RTOL, OUT_ATOL, Case, new_err, to_dev_bits
+from gpu_common import (DEV, LSE_RTOL, OUT_ATOL, Case, assert_attention_close, new_err,
+                        to_dev_bits)
 
 pytestmark = pytest.mark.gpu
 
@@ -42,6 +43,7 @@ def test_static_scratch_matches_caller_workspace(fmt, D, lens):
     assert kvq.kv_decode_workspace_size(fmt, c.B, c.Hq, c.Hkv, D, c.max_blocks * 16) > 0
     ref_out, ref_lse = c.decode()  # regular entry point, caller workspace
     assert int(c.err.item()) == 0
+    ora_out, ora_lse = c.reference()  # the CPU oracle, float64
     for _ in range(2):  # two calls in a row share the one built-in array
         out = torch.full((c.B, c.Hq, D), float("nan"), device=DEV)
         lse = torch.full((c.B, c.Hq), float("nan"), device=DEV)
@@ -50,6 +52,8 @@ def test_static_scratch_matches_caller_workspace(fmt, D, lens):
         torch.cuda.synchronize()
         assert int(err.item()) == 0
         o, l = out.cpu().numpy(), lse.cpu().numpy()
+        # the float64 oracle first, then the regular entry point
+        assert_attention_close(o, l, ora_out, ora_lse)
         assert np.abs(o - ref_out).max() <= OUT_ATOL
         assert (np.abs(l - ref_lse) / np.maximum(np.abs(ref_lse), 1.0)).max() <= LSE_RTOL
 
