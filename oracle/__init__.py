@@ -13,6 +13,8 @@ Sources of each definition (cited by page title and section):
   * "I Tested NVFP4 vs FP8 KV Cache on Blackwell", "What you'll learn": E4M3 at
     one byte per number; NVFP4 = block-scaled 4-bit float with FP8 block
     scales, 4.5 bits per number.
+  * "FP8 KV calibration guide", paragraphs on the calibrator (Q maxima too)
+    and on probability scales: the FP8-attention variant with E4M3 Q and P.
   * OCP 8-bit FP (E4M3) and OCP MX (E2M1) format definitions.
 """
 from __future__ import annotations
@@ -94,6 +96,9 @@ def lib():
         L.orc_prefill_attention.argtypes = [i32, P, P, P, i64, i32, i32, P, i32, P, i32, i32,
                                             i32, f32, f32, f64, P, i64, P, P]
         L.orc_merge.argtypes = [i32, i32, P, P, P, P, P]
+        L.orc_decode_attention_fp8qp.restype = i32
+        L.orc_decode_attention_fp8qp.argtypes = [P, P, P, i64, i32, i32, P, i32, P, i32, i32,
+                                                 f32, f32, f32, f32, f64, f64, P, i64, P, P, P]
         _lib = L
     return _lib
 
@@ -294,3 +299,36 @@ def merge(o_parts, m_parts, l_parts):
     lse = ctypes.c_double()
     lib().orc_merge(n, D, _p(o), _p(m), _p(l), _p(out), ctypes.byref(lse))
     return out, lse.value
+
+
+def decode_attention_fp8qp(q_bits, k_cache, v_cache, H: int, block_table, seq_lens, k_scale,
+                           v_scale, q_scale, prob_scale, sm_scale=None, pairs=None, eps=0.0):
+    """Float64 decode attention with E4M3 Q and E4M3 P over an FP8 cache
+    (orc_decode_attention_fp8qp): Q quantized with q_scale, P quantized page by
+    page relative to the page's largest score with prob_scale.  Returns (out
+    [B][Hq][D], lse [B][Hq], amb [B][Hq]); amb bounds how far out can move if
+    the P codes within relative ``eps`` of a rounding boundary took the other
+    neighbour.  With ``pairs`` only those (b, j) rows are computed."""
+    q = _c(q_bits, np.uint16)
+    B, Hq, D = q.shape
+    bt = _c(block_table, np.int32)
+    sl = _c(seq_lens, np.int32)
+    nb = k_cache.size // (H * head_page_bytes("fp8", D))
+    if sm_scale is None:
+        sm_scale = 1.0 / np.sqrt(D)
+    out = np.full((B, Hq, D), np.nan)
+    lse = np.full((B, Hq), np.nan)
+    amb = np.full((B, Hq), np.nan)
+    if pairs is None:
+        pp, npairs = None, 0
+    else:
+        pr = _c(pairs, np.int32).reshape(-1, 2)
+        pp, npairs = _p(pr), pr.shape[0]
+    rc = lib().orc_decode_attention_fp8qp(_p(q), _p(k_cache), _p(v_cache), nb, H, D, _p(bt),
+                                          bt.shape[1], _p(sl), B, Hq, float(k_scale),
+                                          float(v_scale), float(q_scale), float(prob_scale),
+                                          float(sm_scale), float(eps), pp, npairs, _p(out),
+                                          _p(lse), _p(amb))
+    if rc:
+        raise ValueError(f"oracle fp8 q/p attention failed ({rc})")
+    return out, lse, amb

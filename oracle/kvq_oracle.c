@@ -22,6 +22,10 @@
  *            head_dim, E4M3 block scale = block_absmax / (6 g), FP32 per-tensor
  *            g = tensor_absmax / (448 * 6)) is the recipe this library
  *            implements; the page fixes only the format family and its size.
+ *   [FP8-KV], the paragraphs on the calibrator (it observes Q as well as K and
+ *            V maxima) and on the Q/K/V-only sidecar (other attention paths
+ *            accept probability scales): the FP8-attention variant at the end
+ *            of this file, with E4M3 Q and E4M3 P.
  *   OCP 8-bit floating point specification (E4M3: bias 7, no infinities,
  *            S.1111.111 is NaN, max finite 448) and the OCP MX specification
  *            (E2M1: bias 1, magnitudes 0, .5, 1, 1.5, 2, 3, 4, 6, no NaN/Inf).
@@ -539,4 +543,154 @@ void orc_merge(int n, int D, const double* o_parts, const double* m_parts, const
   }
   for (int d = 0; d < D; d++) out[d] /= L;
   *lse = M + log(L);
+}
+
+/* ------------------------------------------------------------------------ */
+/* FP8 attention over an FP8 cache: E4M3 Q and E4M3 P                       */
+/* ------------------------------------------------------------------------ */
+/*
+ * [FP8-KV], paragraph on the Radiance calibrator: it observes the BF16 Q, K
+ * and V activation maxima and writes per-layer E4M3 scales with the formula of
+ * orc_fp8_scale; and the paragraph on the Q/K/V-only sidecar: other attention
+ * paths also accept a probability scale (prob_scale).  With Q and the softmax
+ * probabilities P in E4M3 as well as K and V, both attention products take
+ * E4M3 operands.  The pages fix no more than that; this is the plain reading
+ * the oracle takes, step by step:
+ *   1. q_hat_d = E4M3(q_d / q_scale)  (fp32 division, RNE, satfinite, as the
+ *      cache write);
+ *   2. s_t = sm_scale * q_scale * k_scale * sum_d dec(q_hat_d) dec(k_{t,d});
+ *   3. P is quantized page by page (the cache's 16-token blocks), relative to
+ *      the page's largest score m_i, so that each page's largest probability
+ *      is 1: p_t = exp(s_t - m_i), p_hat_t = dec(E4M3(p_t / prob_scale)) *
+ *      prob_scale (the decision taken on fp32(p_t) * fp32(1 / prob_scale));
+ *   4. the normaliser uses the unquantized probabilities, and pages merge by
+ *      log-sum-exp: M = max_i m_i,
+ *        out = sum_i exp(m_i - M) sum_{t in i} p_hat_t v_hat_t
+ *              / sum_i exp(m_i - M) sum_{t in i} p_t,
+ *        lse = M + ln(sum_i exp(m_i - M) sum_{t in i} p_t).
+ * Only the FP8 cache format takes this path (its K and V are E4M3 already).
+ *
+ * Where floating point decides a code, the GPU decides on its own fp32 p_t,
+ * which can differ from this float64 p_t in the last bits.  For the checks,
+ * amb (if not NULL) receives per (b, j) row a bound on how far out can move
+ * if every p_t whose fp32(p_t) * fp32(1 / prob_scale) lies within relative
+ * distance eps of an E4M3 rounding boundary took the other neighbouring code:
+ *   amb = sum over such t of exp(m_i - M) * |other - chosen| * prob_scale *
+ *         max_d |v_hat_{t,d}| / L.
+ */
+
+/* The two E4M3 neighbours of a finite x in [0, 448]: lo <= x <= hi (equal
+ * when x is representable). */
+static void e4m3_neighbours(double x, double* lo, double* hi) {
+  double best_lo = 0.0, best_hi = 448.0;
+  for (int c = 0; c <= 0x7E; c++) {
+    double v = (double)orc_e4m3_decode((uint8_t)c);
+    if (v <= x && v > best_lo) best_lo = v;
+    if (v >= x && v < best_hi) best_hi = v;
+  }
+  *lo = best_lo;
+  *hi = best_hi;
+}
+
+int orc_decode_attention_fp8qp(const uint16_t* q, const uint8_t* k_cache, const uint8_t* v_cache,
+                               int64_t num_blocks, int H, int D, const int32_t* block_table,
+                               int max_blocks, const int32_t* seq_lens, int B, int Hq,
+                               float k_scale, float v_scale, float q_scale, float prob_scale,
+                               double sm_scale, double eps, const int32_t* pairs,
+                               int64_t n_pairs, double* out, double* lse, double* amb) {
+  int G = Hq / H;
+  int64_t total = pairs ? n_pairs : (int64_t)B * Hq;
+  float inv_ps = 1.0f / prob_scale;
+  for (int64_t i = 0; i < total; i++) {
+    int b = pairs ? pairs[2 * i] : (int)(i / Hq);
+    int j = pairs ? pairs[2 * i + 1] : (int)(i % Hq);
+    int kv = j / G;
+    int64_t len = seq_lens[b];
+    const uint16_t* q_row = q + ((int64_t)b * Hq + j) * D;
+    const int32_t* bt_row = block_table + (int64_t)b * max_blocks;
+    int64_t row = (int64_t)b * Hq + j;
+    double* o = out + row * D;
+    for (int d = 0; d < D; d++) o[d] = 0.0;
+    if (len <= 0) {
+      lse[row] = -INFINITY;
+      if (amb) amb[row] = 0.0;
+      continue;
+    }
+    double* qh = (double*)malloc(sizeof(double) * (size_t)D);
+    double* s = (double*)malloc(sizeof(double) * (size_t)len);
+    double* w = (double*)malloc(sizeof(double) * (size_t)len);
+    if (!qh || !s || !w) {
+      free(qh);
+      free(s);
+      free(w);
+      return -2;
+    }
+    /* step 1: the quantized query */
+    for (int d = 0; d < D; d++) {
+      float x = bf16_to_f32(q_row[d]) / q_scale;
+      qh[d] = (double)orc_e4m3_decode(orc_e4m3_encode(x));
+    }
+    /* step 2: scores over the E4M3 values */
+    for (int64_t t = 0; t < len; t++) {
+      int64_t blk = bt_row[t / ORC_PAGE];
+      if (blk < 0 || blk >= num_blocks) {
+        free(qh);
+        free(s);
+        free(w);
+        return -1;
+      }
+      int off = (int)(t % ORC_PAGE);
+      const uint8_t* krow = k_cache + ((blk * H + kv) * ORC_PAGE + off) * (int64_t)D;
+      double acc = 0.0;
+      for (int d = 0; d < D; d++) acc += qh[d] * (double)orc_e4m3_decode(krow[d]);
+      s[t] = sm_scale * (double)q_scale * (double)k_scale * acc;
+    }
+    /* M: the largest score (the largest page maximum) */
+    double M = -INFINITY;
+    for (int64_t t = 0; t < len; t++)
+      if (s[t] > M) M = s[t];
+    /* steps 3-4, page by page */
+    double L = 0.0;
+    for (int64_t p0 = 0; p0 < len; p0 += ORC_PAGE) {
+      int64_t p1 = p0 + ORC_PAGE < len ? p0 + ORC_PAGE : len;
+      double mi = -INFINITY;
+      for (int64_t t = p0; t < p1; t++)
+        if (s[t] > mi) mi = s[t];
+      double f = exp(mi - M);
+      for (int64_t t = p0; t < p1; t++) {
+        double p = exp(s[t] - mi);
+        float x = (float)p * inv_ps;
+        uint8_t code = orc_e4m3_encode(x);
+        double chosen = (double)orc_e4m3_decode(code);
+        L += f * p;
+        int64_t blk = bt_row[t / ORC_PAGE];
+        int off = (int)(t % ORC_PAGE);
+        const uint8_t* vrow = v_cache + ((blk * H + kv) * ORC_PAGE + off) * (int64_t)D;
+        double vmax = 0.0;
+        for (int d = 0; d < D; d++) {
+          double v = (double)orc_e4m3_decode(vrow[d]) * (double)v_scale;
+          o[d] += f * chosen * (double)prob_scale * v;
+          if (fabs(v) > vmax) vmax = fabs(v);
+        }
+        /* a rounding boundary within relative eps of x: the other neighbour
+         * is a possible code too */
+        double lo, hi;
+        e4m3_neighbours((double)x, &lo, &hi);
+        double other = chosen == lo ? hi : lo;
+        int near = (double)x < 448.0 && fabs((double)x - 0.5 * (lo + hi)) <= eps * (double)x;
+        w[t] = near ? f * fabs(other - chosen) * (double)prob_scale * vmax : 0.0;
+      }
+    }
+    for (int d = 0; d < D; d++) o[d] /= L;
+    lse[row] = M + log(L);
+    if (amb) {
+      double a = 0.0;
+      for (int64_t t = 0; t < len; t++) a += w[t];
+      amb[row] = a / L;
+    }
+    free(qh);
+    free(s);
+    free(w);
+  }
+  return 0;
 }
