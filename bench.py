@@ -570,6 +570,19 @@ def main():
         del s1
         torch.cuda.empty_cache()
 
+        # FP8 attention (E4M3 q and P, both products on E4M3 tensor cores) on
+        # the FP8 caches of the agent and the 1 x 65,536-token workloads
+        fq = {}
+        for key, name in (("4x127k", "agents-fp8-4x127k"), ("1x64k", "nvfp4-1x64k")):
+            s4 = DecodeScenario(wl.WORKLOADS[name], fmt="fp8", device="cuda")
+            s4.fp8qp_setup()
+            (dms,), _ = timer.run([s4.decode_fp8qp], Kx, W)
+            assert int(s4.err.item()) == 0
+            fq[key] = row(s4.scan_bytes, dms, peak)
+            del s4
+            torch.cuda.empty_cache()
+        extras["fp8_attention"] = fq
+
         # BF16 vs FP8 vs NVFP4 decode on the byte-heavy 4 x 126,976-token
         # D=128 cache and on the 1 x 65,536-token D=64 workload
         for key, name, reps in (("formats_4x127k", "agents-fp8-4x127k", Kx),

@@ -233,6 +233,38 @@ kvq_status kv_decode_attention_window(int32_t fmt, const void* q, const kvq_cach
                                       float* lse, void* workspace, size_t workspace_bytes,
                                       int32_t* d_err, kvq_stream stream);
 
+/* FP8 attention over an FP8 cache: kv_decode_attention with the query and the
+ * softmax probabilities in E4M3 too, so both attention products run on E4M3
+ * tensor cores ("FP8 KV calibration guide": the calibrator observes the BF16
+ * Q, K and V activation maxima and writes per-layer E4M3 scales with the same
+ * formula, and other attention paths accept a probability scale, prob_scale).
+ *   d_q_scale    : device fp32 scalar, the query's E4M3 scale (the per-layer
+ *                  formula of kv_scale_from_absmax on Q's abs-max):
+ *                  q_hat = E4M3(q / q_scale) (fp32 division, nearest even,
+ *                  saturating).
+ *   d_prob_scale : device fp32 scalar, P's E4M3 scale (the same formula at an
+ *                  observed maximum of 1 gives 1.05 / 448).
+ * P is quantized page by page: within each 16-token cache page the
+ * probabilities are taken against the page's largest score (so each page's
+ * largest p is 1), P_hat = E4M3(p * fp32(1 / prob_scale)); the page then
+ * enters the softmax sums with weight exp(page max - running max), and the
+ * normaliser uses the unquantized p.  Results therefore differ from
+ * kv_decode_attention by the E4M3 rounding of q and of P (about 2^-4
+ * relative per probability); the split over CTAs does not change them.
+ * Other arguments, layouts, the workspace (kv_decode_workspace_size with
+ * KVQ_FMT_FP8_E4M3 and the same sizes) and the errors are those of
+ * kv_decode_attention.  The cache must be FP8 (KVQ_ERR_UNSUPPORTED
+ * otherwise); d_q_scale / d_prob_scale NULL is KVQ_ERR_INVALID_ARG, and a
+ * non-positive or non-finite value on the device sets KVQ_DERR_SCALE. */
+kvq_status kv_decode_attention_fp8qp(const void* q, const kvq_cache* cache,
+                                     const int32_t* block_table, int32_t max_blocks,
+                                     const int32_t* seq_lens, int32_t num_seqs,
+                                     int32_t num_q_heads, int32_t max_seq_len, int32_t num_splits,
+                                     const float* d_k_scale, const float* d_v_scale,
+                                     const float* d_q_scale, const float* d_prob_scale,
+                                     float sm_scale, float* out, float* lse, void* workspace,
+                                     size_t workspace_bytes, int32_t* d_err, kvq_stream stream);
+
 /* Workspace bytes kv_decode_attention_window needs (as
  * kv_decode_workspace_size, with the window). */
 kvq_status kv_decode_workspace_size_window(int32_t fmt, int32_t num_seqs, int32_t num_q_heads,

@@ -306,9 +306,10 @@ def decode_attention_fp8qp(q_bits, k_cache, v_cache, H: int, block_table, seq_le
     """Float64 decode attention with E4M3 Q and E4M3 P over an FP8 cache
     (orc_decode_attention_fp8qp): Q quantized with q_scale, P quantized page by
     page relative to the page's largest score with prob_scale.  Returns (out
-    [B][Hq][D], lse [B][Hq], amb [B][Hq]); amb bounds how far out can move if
-    the P codes within relative ``eps`` of a rounding boundary took the other
-    neighbour.  With ``pairs`` only those (b, j) rows are computed."""
+    [B][Hq][D], lse [B][Hq], amb [B][Hq][D]); amb bounds how far each output
+    can move if the P codes within relative ``eps`` of a rounding boundary
+    took the other neighbour.  With ``pairs`` only those (b, j) rows are
+    computed."""
     q = _c(q_bits, np.uint16)
     B, Hq, D = q.shape
     bt = _c(block_table, np.int32)
@@ -318,7 +319,7 @@ def decode_attention_fp8qp(q_bits, k_cache, v_cache, H: int, block_table, seq_le
         sm_scale = 1.0 / np.sqrt(D)
     out = np.full((B, Hq, D), np.nan)
     lse = np.full((B, Hq), np.nan)
-    amb = np.full((B, Hq), np.nan)
+    amb = np.full((B, Hq, D), np.nan)
     if pairs is None:
         pp, npairs = None, 0
     else:

@@ -572,11 +572,12 @@ void orc_merge(int n, int D, const double* o_parts, const double* m_parts, const
  *
  * Where floating point decides a code, the GPU decides on its own fp32 p_t,
  * which can differ from this float64 p_t in the last bits.  For the checks,
- * amb (if not NULL) receives per (b, j) row a bound on how far out can move
- * if every p_t whose fp32(p_t) * fp32(1 / prob_scale) lies within relative
- * distance eps of an E4M3 rounding boundary took the other neighbouring code:
- *   amb = sum over such t of exp(m_i - M) * |other - chosen| * prob_scale *
- *         max_d |v_hat_{t,d}| / L.
+ * amb (if not NULL, [B][Hq][D] like out) receives a bound on how far each
+ * output can move if every p_t whose fp32(p_t) * fp32(1 / prob_scale) lies
+ * within relative distance eps of an E4M3 rounding boundary took the other
+ * neighbouring code:
+ *   amb_d = sum over such t of exp(m_i - M) * |other - chosen| * prob_scale *
+ *           |v_hat_{t,d}| / L.
  */
 
 /* The two E4M3 neighbours of a finite x in [0, 448]: lo <= x <= hi (equal
@@ -611,9 +612,10 @@ int orc_decode_attention_fp8qp(const uint16_t* q, const uint8_t* k_cache, const 
     int64_t row = (int64_t)b * Hq + j;
     double* o = out + row * D;
     for (int d = 0; d < D; d++) o[d] = 0.0;
+    if (amb)
+      for (int d = 0; d < D; d++) amb[row * D + d] = 0.0;
     if (len <= 0) {
       lse[row] = -INFINITY;
-      if (amb) amb[row] = 0.0;
       continue;
     }
     double* qh = (double*)malloc(sizeof(double) * (size_t)D);
@@ -666,11 +668,9 @@ int orc_decode_attention_fp8qp(const uint16_t* q, const uint8_t* k_cache, const 
         int64_t blk = bt_row[t / ORC_PAGE];
         int off = (int)(t % ORC_PAGE);
         const uint8_t* vrow = v_cache + ((blk * H + kv) * ORC_PAGE + off) * (int64_t)D;
-        double vmax = 0.0;
         for (int d = 0; d < D; d++) {
           double v = (double)orc_e4m3_decode(vrow[d]) * (double)v_scale;
           o[d] += f * chosen * (double)prob_scale * v;
-          if (fabs(v) > vmax) vmax = fabs(v);
         }
         /* a rounding boundary within relative eps of x: the other neighbour
          * is a possible code too */
@@ -678,16 +678,20 @@ int orc_decode_attention_fp8qp(const uint16_t* q, const uint8_t* k_cache, const 
         e4m3_neighbours((double)x, &lo, &hi);
         double other = chosen == lo ? hi : lo;
         int near = (double)x < 448.0 && fabs((double)x - 0.5 * (lo + hi)) <= eps * (double)x;
-        w[t] = near ? f * fabs(other - chosen) * (double)prob_scale * vmax : 0.0;
+        w[t] = near ? f * fabs(other - chosen) * (double)prob_scale : 0.0;
       }
     }
     for (int d = 0; d < D; d++) o[d] /= L;
     lse[row] = M + log(L);
-    if (amb) {
-      double a = 0.0;
-      for (int64_t t = 0; t < len; t++) a += w[t];
-      amb[row] = a / L;
-    }
+    if (amb)
+      for (int64_t t = 0; t < len; t++) {
+        if (w[t] == 0.0) continue;
+        int64_t blk = bt_row[t / ORC_PAGE];
+        int off = (int)(t % ORC_PAGE);
+        const uint8_t* vrow = v_cache + ((blk * H + kv) * ORC_PAGE + off) * (int64_t)D;
+        for (int d = 0; d < D; d++)
+          amb[row * D + d] += w[t] * fabs((double)orc_e4m3_decode(vrow[d]) * (double)v_scale) / L;
+      }
     free(qh);
     free(s);
     free(w);

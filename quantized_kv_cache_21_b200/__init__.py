@@ -33,6 +33,7 @@ EXPORTS = ("kvq_status_string", "kvq_last_error", "kv_cache_bytes", "kv_scale_fr
            "kv_scale_from_absmax_device", "kv_calibrate_absmax", "kv_quantize_write",
            "kv_decode_workspace_size", "kv_decode_attention", "kv_decode_attention_static_ws",
            "kv_decode_attention_window", "kv_decode_workspace_size_window",
+           "kv_decode_attention_fp8qp",
            "kv_prefill_attention", "kv_dequantize", "kvq_selftest_bounded_wait")
 
 
@@ -78,6 +79,8 @@ def lib() -> ctypes.CDLL:
                                            f32, P, P, P, sz, P, P],
             "kv_decode_workspace_size_window": [i32, i32, i32, i32, i32, i32, i32, i32,
                                                 ctypes.POINTER(sz)],
+            "kv_decode_attention_fp8qp": [P, CP, P, i32, P, i32, i32, i32, i32, P, P, P, P, f32,
+                                          P, P, P, sz, P, P],
             "kv_prefill_attention": [i32, P, CP, P, i32, P, i32, i32, i32, P, P, f32, P, P, P,
                                      P],
             "kv_dequantize": [i32, CP, P, i64, P, P, P, P, P, P],
@@ -259,6 +262,27 @@ def kv_decode_attention_window(fmt, q: torch.Tensor, cache: KVCache, block_table
                                             _ptr(v_scale), float(sm_scale), _ptr(out), _ptr(lse),
                                             _ptr(workspace), ws_bytes, _ptr(d_err),
                                             _stream(stream)))
+
+
+def kv_decode_attention_fp8qp(q: torch.Tensor, cache: KVCache, block_table: torch.Tensor,
+                              seq_lens: torch.Tensor, max_seq_len: int, k_scale, v_scale,
+                              q_scale, prob_scale, out: torch.Tensor, lse: torch.Tensor | None,
+                              workspace: torch.Tensor | None, d_err: torch.Tensor | None = None,
+                              sm_scale: float = 0.0, num_splits: int = 0, stream=None):
+    """FP8 attention over an FP8 cache: q and the softmax probabilities in
+    E4M3 too (q_scale, prob_scale: device fp32 scalars; see include/kvq.h).
+    Shapes and the workspace as kv_decode_attention with the "fp8" format."""
+    assert q.dtype == torch.bfloat16 and q.is_contiguous()
+    assert block_table.dtype == torch.int32 and seq_lens.dtype == torch.int32
+    assert out.dtype == torch.float32
+    B, Hq, _ = q.shape
+    ws_bytes = workspace.numel() if workspace is not None else 0
+    _check(lib().kv_decode_attention_fp8qp(_ptr(q), cache.c, _ptr(block_table),
+                                           block_table.shape[1], _ptr(seq_lens), B, Hq,
+                                           max_seq_len, num_splits, _ptr(k_scale), _ptr(v_scale),
+                                           _ptr(q_scale), _ptr(prob_scale), float(sm_scale),
+                                           _ptr(out), _ptr(lse), _ptr(workspace), ws_bytes,
+                                           _ptr(d_err), _stream(stream)))
 
 
 def kv_prefill_attention(fmt, q: torch.Tensor, cache: KVCache, block_table: torch.Tensor,

@@ -154,8 +154,18 @@ kvq_status encode(CUtensorMap* m, CUtensorMapDataType dt, cuuint32_t rank, void*
   auto fn = encode_fn();
   if (!fn) return fail(KVQ_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
   const cuuint32_t es[5] = {1, 1, 1, 1, 1};
-  CUresult r = fn(m, dt, rank, base, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
-                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  auto call = [&] {
+    return fn(m, dt, rank, base, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  };
+  CUresult r = call();
+  if (r == CUDA_ERROR_INVALID_CONTEXT) {
+    // A host thread that has made no CUDA runtime call yet has no current
+    // context, and the encoder (a driver call) needs one: make the current
+    // device's primary context current, as the runtime's own launch would.
+    int dev = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess && cudaSetDevice(dev) == cudaSuccess) r = call();
+  }
   if (r != CUDA_SUCCESS) return fail(KVQ_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
   return KVQ_OK;
 }
@@ -409,14 +419,19 @@ kvq_status kv_decode_attention(int32_t fmt, const void* q, const kvq_cache* cach
                                     sm_scale, out, lse, workspace, workspace_bytes, d_err, stream);
 }
 
-kvq_status kv_decode_attention_window(int32_t fmt, const void* q, const kvq_cache* cache,
-                                      const int32_t* block_table, int32_t max_blocks,
-                                      const int32_t* seq_lens, int32_t num_seqs,
-                                      int32_t num_q_heads, int32_t max_seq_len, int32_t window,
-                                      int32_t num_splits, const float* d_k_scale,
-                                      const float* d_v_scale, float sm_scale, float* out,
-                                      float* lse, void* workspace, size_t workspace_bytes,
-                                      int32_t* d_err, kvq_stream stream) {
+}  // extern "C"
+
+namespace {
+// The decode launches behind kv_decode_attention, its window mode and its FP8
+// attention variant (d_q_scale / d_prob_scale non-NULL: E4M3 Q and P).
+kvq_status decode_impl(int32_t fmt, const void* q, const kvq_cache* cache,
+                       const int32_t* block_table, int32_t max_blocks, const int32_t* seq_lens,
+                       int32_t num_seqs, int32_t num_q_heads, int32_t max_seq_len, int32_t window,
+                       int32_t num_splits, const float* d_k_scale, const float* d_v_scale,
+                       const float* d_q_scale, const float* d_prob_scale, float sm_scale,
+                       float* out, float* lse, void* workspace, size_t workspace_bytes,
+                       int32_t* d_err, kvq_stream stream) {
+  const bool qp = d_q_scale || d_prob_scale;
   kvq_status s = check_cache(fmt, cache);
   if (s != KVQ_OK) return s;
   const int D = cache->head_dim, Hkv = cache->num_kv_heads;
@@ -431,6 +446,13 @@ kvq_status kv_decode_attention_window(int32_t fmt, const void* q, const kvq_cach
     return fail(KVQ_ERR_INVALID_ARG, "max_seq_len %d exceeds max_blocks * 16", max_seq_len);
   if (fmt != KVQ_FMT_BF16 && (!d_k_scale || !d_v_scale))
     return fail(KVQ_ERR_INVALID_ARG, "quantized formats need d_k_scale and d_v_scale");
+  if (qp) {
+    if (fmt != KVQ_FMT_FP8_E4M3)
+      return fail(KVQ_ERR_UNSUPPORTED, "FP8 attention needs an FP8 cache (format %d given)", fmt);
+    if (!d_q_scale || !d_prob_scale)
+      return fail(KVQ_ERR_INVALID_ARG, "FP8 attention needs d_q_scale and d_prob_scale");
+    if (window != 0) return fail(KVQ_ERR_UNSUPPORTED, "FP8 attention has no window mode");
+  }
   if (sm_scale == 0.0f) sm_scale = 1.0f / sqrtf((float)D);
   if (!isfinite(sm_scale)) return fail(KVQ_ERR_INVALID_ARG, "sm_scale not finite");
   s = check_device();
@@ -456,6 +478,8 @@ kvq_status kv_decode_attention_window(int32_t fmt, const void* q, const kvq_cach
   p.seq_lens = seq_lens;
   p.k_scale = d_k_scale;
   p.v_scale = d_v_scale;
+  p.q_scale = d_q_scale;
+  p.prob_scale = d_prob_scale;
   p.out = out;
   p.lse = lse;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
@@ -474,8 +498,43 @@ kvq_status kv_decode_attention_window(int32_t fmt, const void* q, const kvq_cach
   p.max_seq_len = max_seq_len;
   p.window = window;
   p.sm_scale = sm_scale;
-  cudaError_t e = kvq::launch_decode(fmt, D, maps, p, pl.ctas, static_cast<cudaStream_t>(stream));
+  cudaError_t e =
+      kvq::launch_decode(fmt, D, maps, p, pl.ctas, static_cast<cudaStream_t>(stream), qp);
   return e == cudaSuccess ? KVQ_OK : cuda_fail(e, "decode kernel");
+}
+}  // namespace
+
+extern "C" {
+
+kvq_status kv_decode_attention_window(int32_t fmt, const void* q, const kvq_cache* cache,
+                                      const int32_t* block_table, int32_t max_blocks,
+                                      const int32_t* seq_lens, int32_t num_seqs,
+                                      int32_t num_q_heads, int32_t max_seq_len, int32_t window,
+                                      int32_t num_splits, const float* d_k_scale,
+                                      const float* d_v_scale, float sm_scale, float* out,
+                                      float* lse, void* workspace, size_t workspace_bytes,
+                                      int32_t* d_err, kvq_stream stream) {
+  return decode_impl(fmt, q, cache, block_table, max_blocks, seq_lens, num_seqs, num_q_heads,
+                     max_seq_len, window, num_splits, d_k_scale, d_v_scale, nullptr, nullptr,
+                     sm_scale, out, lse, workspace, workspace_bytes, d_err, stream);
+}
+
+kvq_status kv_decode_attention_fp8qp(const void* q, const kvq_cache* cache,
+                                     const int32_t* block_table, int32_t max_blocks,
+                                     const int32_t* seq_lens, int32_t num_seqs,
+                                     int32_t num_q_heads, int32_t max_seq_len, int32_t num_splits,
+                                     const float* d_k_scale, const float* d_v_scale,
+                                     const float* d_q_scale, const float* d_prob_scale,
+                                     float sm_scale, float* out, float* lse, void* workspace,
+                                     size_t workspace_bytes, int32_t* d_err, kvq_stream stream) {
+  if (cache && cache->fmt != KVQ_FMT_FP8_E4M3)
+    return fail(KVQ_ERR_UNSUPPORTED, "FP8 attention needs an FP8 cache (format %d given)",
+                cache->fmt);
+  if (!d_q_scale || !d_prob_scale)
+    return fail(KVQ_ERR_INVALID_ARG, "FP8 attention needs d_q_scale and d_prob_scale");
+  return decode_impl(KVQ_FMT_FP8_E4M3, q, cache, block_table, max_blocks, seq_lens, num_seqs,
+                     num_q_heads, max_seq_len, 0, num_splits, d_k_scale, d_v_scale, d_q_scale,
+                     d_prob_scale, sm_scale, out, lse, workspace, workspace_bytes, d_err, stream);
 }
 
 kvq_status kv_prefill_attention(int32_t fmt, const void* q, const kvq_cache* cache,

@@ -100,14 +100,15 @@ struct Fmt<1, 128> {
   struct Raw {
     uint4 k[4], v[4];
   };
-  static constexpr bool kLateV = false;
-  __device__ static void load_raw(const uint8_t* st, int gid, int tig, Raw& r) {
+  __device__ static void load_raw_k(const uint8_t* st, int gid, int tig, Raw& r) {
 #pragma unroll
     for (int rr = 0; rr < 2; ++rr) {
       const int row = gid + 8 * rr;
       r.k[2 * rr] = lds128(st + swz128(row, 32 * tig));
       r.k[2 * rr + 1] = lds128(st + swz128(row, 32 * tig + 16));
     }
+  }
+  __device__ static void load_raw_v(const uint8_t* st, int gid, int tig, Raw& r) {
     const uint8_t* sv = st + V_OFF;
     r.v[0] = lds128(sv + swz128(2 * tig, 16 * gid));
     r.v[1] = lds128(sv + swz128(2 * tig + 1, 16 * gid));
@@ -159,10 +160,11 @@ struct Fmt<1, 64> {
     uint4 k[2];
     uint2 v[4];
   };
-  static constexpr bool kLateV = false;
-  __device__ static void load_raw(const uint8_t* st, int gid, int tig, Raw& r) {
+  __device__ static void load_raw_k(const uint8_t* st, int gid, int tig, Raw& r) {
 #pragma unroll
     for (int rr = 0; rr < 2; ++rr) r.k[rr] = lds128(st + swz64(gid + 8 * rr, 16 * tig));
+  }
+  __device__ static void load_raw_v(const uint8_t* st, int gid, int tig, Raw& r) {
     const uint8_t* sv = st + V_OFF;
     r.v[0] = lds64(sv + swz64(2 * tig, 8 * gid));
     r.v[1] = lds64(sv + swz64(2 * tig + 1, 8 * gid));
@@ -212,14 +214,15 @@ struct Fmt<0, 64> {
   struct Raw {
     uint4 k[4], v[4];
   };
-  static constexpr bool kLateV = false;
-  __device__ static void load_raw(const uint8_t* st, int gid, int tig, Raw& r) {
+  __device__ static void load_raw_k(const uint8_t* st, int gid, int tig, Raw& r) {
 #pragma unroll
     for (int rr = 0; rr < 2; ++rr) {
       const int row = gid + 8 * rr;
       r.k[2 * rr] = lds128(st + swz128(row, 32 * tig));
       r.k[2 * rr + 1] = lds128(st + swz128(row, 32 * tig + 16));
     }
+  }
+  __device__ static void load_raw_v(const uint8_t* st, int gid, int tig, Raw& r) {
     const uint8_t* sv = st + V_OFF;
     r.v[0] = lds128(sv + swz128(2 * tig, 16 * gid));
     r.v[1] = lds128(sv + swz128(2 * tig + 1, 16 * gid));
@@ -281,9 +284,6 @@ struct Fmt<0, 128> {
   struct Raw {
     uint4 k[8], v[8];
   };
-  // 64 raw registers would not fit beside the accumulators: K is read and
-  // used first, V read after the QK product (kLateV), then the stage refilled.
-  static constexpr bool kLateV = true;
   __device__ static void load_raw_k(const uint8_t* st, int gid, int tig, Raw& r) {
 #pragma unroll
     for (int hf = 0; hf < 2; ++hf) {
@@ -379,14 +379,15 @@ struct Fmt<2, 64> {
     uint2 k[2];
     uint32_t v[4], ks[2], vs[4];
   };
-  static constexpr bool kLateV = false;
-  __device__ static void load_raw(const uint8_t* st, int gid, int tig, Raw& r) {
+  __device__ static void load_raw_k(const uint8_t* st, int gid, int tig, Raw& r) {
 #pragma unroll
     for (int rr = 0; rr < 2; ++rr) {
       const int row = gid + 8 * rr;
       r.k[rr] = lds64(st + swz32(row, 8 * tig));
       r.ks[rr] = st[KSF + row * 4 + tig];
     }
+  }
+  __device__ static void load_raw_v(const uint8_t* st, int gid, int tig, Raw& r) {
     const uint8_t* sv = st + V_OFF;
     const uint8_t* ss = st + VSF;
     const int t0 = 2 * tig, t2 = 2 * tig + 8, blk = gid >> 1;
@@ -464,14 +465,15 @@ struct Fmt<2, 128> {
     uint2 v[4];
     uint32_t ks[2], vs[4];
   };
-  static constexpr bool kLateV = false;
-  __device__ static void load_raw(const uint8_t* st, int gid, int tig, Raw& r) {
+  __device__ static void load_raw_k(const uint8_t* st, int gid, int tig, Raw& r) {
 #pragma unroll
     for (int rr = 0; rr < 2; ++rr) {
       const int row = gid + 8 * rr;
       r.k[rr] = lds128(st + swz64(row, 16 * tig));
       r.ks[rr] = *reinterpret_cast<const uint16_t*>(st + KSF + row * 8 + 2 * tig);
     }
+  }
+  __device__ static void load_raw_v(const uint8_t* st, int gid, int tig, Raw& r) {
     const uint8_t* sv = st + V_OFF;
     const uint8_t* ss = st + VSF;
     const int t0 = 2 * tig, t2 = 2 * tig + 8;
@@ -704,7 +706,7 @@ __device__ __forceinline__ void final_merge(const DecodeParams& p, int u, int b,
   }
 }
 
-template <int FMT, int D>
+template <int FMT, int D, bool QP>
 __global__ void __launch_bounds__(Shape<FMT, D>::NW * 32, 1)
     kvq_decode_kernel(const __grid_constant__ CUtensorMap mk, const __grid_constant__ CUtensorMap mv,
                       const __grid_constant__ CUtensorMap mks,
@@ -761,34 +763,69 @@ __global__ void __launch_bounds__(Shape<FMT, D>::NW * 32, 1)
       scale_ok = ks >= 0.f && vs >= 0.f && ks < kInf && vs < kInf;
     if (!scale_ok && c == 0 && tid == 0) set_err(p.d_err, kErrScale);
   }
+  // FP8 attention: the E4M3 scales of q and P (both > 0 and finite).  The
+  // output takes prob_scale, and the 2^kPLog2 that l carries (see pv_page).
+  float qs = 1.f, inv_ps = 1.f, vs_out = vs;
+  if constexpr (QP) {
+    qs = __ldg(p.q_scale);
+    const float ps = __ldg(p.prob_scale);
+    const bool ok = qs > 0.f && qs < kInf && ps > 0.f && ps < kInf;
+    if (!ok) {
+      if (scale_ok && c == 0 && tid == 0) set_err(p.d_err, kErrScale);
+      scale_ok = false;
+    }
+    inv_ps = __fdiv_rn(1.f, ps);
+    vs_out = vs * ps * 4096.f;  // 2^kPLog2
+  }
 
   // Scores are scaled by c = sm_scale * k_scale * log2(e) in the softmax
   // below, and masked tokens carry a raw score of -inf, so c must be positive:
   // a negative sm_scale is moved into Q's sign (exact), and c = 0 (an all-zero
   // NVFP4 K tensor, g = 0, whose scores are all 0) becomes a tiny positive c
   // with the same result.
-  const float c_raw = p.sm_scale * ks * kLog2e;
-  const uint32_t q_sign = c_raw < 0.f ? 0x80008000u : 0u;
+  const float c_raw = p.sm_scale * qs * ks * kLog2e;
+  const uint32_t q_sign = c_raw < 0.f ? (QP ? 0x80808080u : 0x80008000u) : 0u;
   const float c_log2 = fmaxf(fabsf(c_raw), 1e-30f);
 
   // Query fragments (B operand of QK) of unit u; padded heads are 0.  The
   // thread's head-dim elements come in 16-byte runs of 8.
   uint32_t qb[KS][2];
+  // FP8 attention: the E4M3 query as the A operand of QK (rows = heads, row
+  // gid; the padding rows gid+8 are zero): per 32-element k-step s, a0 holds
+  // head-dim elements k_elem(tig, 8s .. 8s+3) and a2 elements 8s+4 .. 8s+7.
+  uint32_t qa[QP ? D / 32 : 1][2];
   auto load_q = [&](int u) {
     const int grp = u % p.n_groups, h = (u / p.n_groups) % p.Hkv, b = u / (p.n_groups * p.Hkv);
     const int qi = grp * 8 + gid;
     const bool hv = qi < p.G;
     const uint16_t* qrow = p.q + (static_cast<size_t>(b) * p.Hq + h * p.G + (hv ? qi : 0)) * D;
+    if constexpr (QP) {
+      // q_hat = E4M3(q / q_scale): IEEE fp32 division, round to nearest even,
+      // saturating (the rounding of the cache write)
 #pragma unroll
-    for (int i = 0; i < D / 4; i += 8) {
-      const uint4 w = hv ? __ldg(reinterpret_cast<const uint4*>(qrow + F::k_elem(tig, i)))
-                         : make_uint4(0u, 0u, 0u, 0u);
-      const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+      for (int s = 0; s < D / 32; ++s) {
+        const uint4 w = hv ? __ldg(reinterpret_cast<const uint4*>(qrow + F::k_elem(tig, 8 * s)))
+                           : make_uint4(0u, 0u, 0u, 0u);
+        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+        uint32_t e[4];
 #pragma unroll
-      for (int x = 0; x < 4; ++x) {
-        uint32_t v = ws[x];
-        if constexpr (!F::kBF16) v = pack_f16x2(bf16_lo(v), bf16_hi(v));
-        qb[i / 4 + x / 2][x & 1] = v ^ q_sign;
+        for (int x = 0; x < 4; ++x)
+          e[x] = f32x2_to_e4m3x2(__fdiv_rn(bf16_lo(ws[x]), qs), __fdiv_rn(bf16_hi(ws[x]), qs));
+        qa[s][0] = (e[0] | (e[1] << 16)) ^ q_sign;
+        qa[s][1] = (e[2] | (e[3] << 16)) ^ q_sign;
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < D / 4; i += 8) {
+        const uint4 w = hv ? __ldg(reinterpret_cast<const uint4*>(qrow + F::k_elem(tig, i)))
+                           : make_uint4(0u, 0u, 0u, 0u);
+        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int x = 0; x < 4; ++x) {
+          uint32_t v = ws[x];
+          if constexpr (!F::kBF16) v = pack_f16x2(bf16_lo(v), bf16_hi(v));
+          qb[i / 4 + x / 2][x & 1] = v ^ q_sign;
+        }
       }
     }
   };
@@ -882,6 +919,16 @@ __global__ void __launch_bounds__(Shape<FMT, D>::NW * 32, 1)
   // no data.
   unsigned ok_win = __ballot_sync(0xffffffffu, cur_blk >= 0 && cur_blk < p.num_blocks);
   unsigned stage_ok = 0;
+  // A stage whose block id is bad gets no copy: the warp zero-fills it (so no
+  // stale or unwritten bytes, possibly NaN codes, reach the V product) and
+  // completes its phase by hand; the page's scores are masked, so it carries
+  // no weight.
+  auto fill_bad = [&](int stg) {
+    uint4* z = reinterpret_cast<uint4*>(ring + stg * F::STAGE);
+#pragma unroll 1
+    for (int i = lane; i < F::STAGE / 16; i += 32) z[i] = make_uint4(0u, 0u, 0u, 0u);
+    __syncwarp();
+  };
   auto issue = [&](int i, int stg) {
     if (i >= chunk + 32) {  // slide the id window by 32 items
       chunk += 32;
@@ -893,6 +940,7 @@ __global__ void __launch_bounds__(Shape<FMT, D>::NW * 32, 1)
     const int src = i - chunk;
     const unsigned ok = (ok_win >> src) & 1u;
     stage_ok = (stage_ok & ~(1u << stg)) | (ok << stg);
+    if (!ok) fill_bad(stg);  // warp-uniform (ok comes from a ballot)
     if (lane == src) {
       uint64_t* bar = &bars[stg];
       fence_proxy_async_smem();  // the warp's reads of this stage precede the copy
@@ -900,28 +948,108 @@ __global__ void __launch_bounds__(Shape<FMT, D>::NW * 32, 1)
         F::issue(ring + stg * F::STAGE, bar, &mk, &mv, &mks, &mvs, cur_h, cur_blk);
       } else {
         set_err(p.d_err, kErrBlockId);
-        mbar_arrive(bar);  // completes the phase with no data; the page is skipped
+        mbar_arrive(bar);  // completes the phase with no data
       }
     }
   };
   // Prologue: lane i fills stage i with local item i (its own cur_blk), the
   // lanes' copies issued together rather than one after another.
+  int issued = min(NSW, n_local);  // local items whose copies have been issued
   {
-    const int n0 = min(NSW, n_local);
-    stage_ok = ok_win & ((1u << n0) - 1u);
-    if (lane < n0) {
+    stage_ok = ok_win & ((1u << issued) - 1u);
+    for (int i = 0; i < issued; ++i)  // rare: zero-fill the stages of bad ids
+      if (!((ok_win >> i) & 1u)) fill_bad(i);
+    if (lane < issued) {
       uint64_t* bar = &bars[lane];
       if ((ok_win >> lane) & 1u) {
         F::issue(ring + lane * F::STAGE, bar, &mk, &mv, &mks, &mvs, cur_h, cur_blk);
       } else {
         set_err(p.d_err, kErrBlockId);
-        mbar_arrive(bar);  // completes the phase with no data; the page is skipped
+        mbar_arrive(bar);  // completes the phase with no data
       }
     }
   }
 
-  int k_base = 0, j = 0;  // j = this warp's next local item
+  // Ring of the warp's local items: item i sits in stage i % NSW and its copy
+  // completes barrier phase (i / NSW) & 1.  A stage is held from the wait for
+  // its item until that item's V has been read, one loop trip later, and is
+  // then refilled with the next item not yet issued.
+  int k_base = 0, j = 0;  // j = this warp's next local item to wait for
   int st = 0, ph = 0;     // its stage (j % NSW) and barrier phase parity ((j / NSW) & 1)
+  bool dead = false;      // a bounded wait expired: this warp reads no more pages
+  // Waits for item j (all lanes agree, so the warp stays converged).  If the
+  // wait expires: report it, wait (bounded) for the copies still in flight
+  // (items j+1 .. issued-1) and stop reading pages.
+  auto wait_item = [&]() -> bool {
+    if (__all_sync(0xffffffffu, mbar_wait_bounded(&bars[st], ph))) return true;
+    if (lane == 0) set_err(p.d_err, kErrTimeout);
+    for (int i = j + 1; i < issued; ++i) mbar_wait_bounded(&bars[i % NSW], (i / NSW) & 1);
+    dead = true;
+    return false;
+  };
+  auto advance = [&]() {
+    ++j;
+    if (++st == NSW) {
+      st = 0;
+      ph ^= 1;
+    }
+  };
+  // Refill the stage of a consumed item with the next item not yet issued.
+  auto refill = [&](int stg) {
+    __syncwarp();  // every lane's reads of the stage are done
+    if (issued < n_local) {
+      issue(issued, stg);
+      ++issued;
+    }
+  };
+  // S^T = K Q^T of the page in stage stg on tensor cores (two accumulator
+  // chains): the raw scores r[i] = q . k_code of this thread's (token, head)
+  // pairs (tokens gid, gid+8; heads 2tig, 2tig+1).
+  // FP8 attention: S[head][token] = Q_hat K^T on E4M3 tensor cores, the K
+  // codes read straight from the stage as the B operand (column = token gid
+  // for tokens 0-7, gid+8 for tokens 8-15); this thread gets head gid's
+  // scores of tokens 2tig, 2tig+1 (r[0], r[1]) and 2tig+8, 2tig+9 (r[2], r[3]).
+  auto qk_page = [&](int stg, float r[4]) {
+    typename F::Raw raw;
+    F::load_raw_k(ring + stg * F::STAGE, gid, tig, raw);
+    if constexpr (QP) {
+      constexpr int NR = sizeof(raw.k) / sizeof(raw.k[0]) / 2;  // uint4 per row
+      float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {  // n-tile t: tokens 8t .. 8t+7, this thread's row gid + 8t
+        uint32_t w[4 * NR];
+#pragma unroll
+        for (int i = 0; i < NR; ++i) {
+          const uint4 x = raw.k[NR * t + i];
+          w[4 * i] = x.x;
+          w[4 * i + 1] = x.y;
+          w[4 * i + 2] = x.z;
+          w[4 * i + 3] = x.w;
+        }
+#pragma unroll
+        for (int s = 0; s < D / 32; ++s)
+          mma_e4m3_k32(t ? s1 : s0, qa[s][0], 0u, qa[s][1], 0u, w[2 * s], w[2 * s + 1]);
+      }
+      r[0] = s0[0];
+      r[1] = s0[1];
+      r[2] = s1[0];
+      r[3] = s1[1];
+      return;
+    }
+    uint32_t ka[KS][4];
+    F::conv_k(raw, ka);
+    float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int s = 0; s < KS; ++s) {
+      if (s & 1)
+        mma16816<F::kBF16>(sb, ka[s], qb[s][0], qb[s][1]);
+      else
+        mma16816<F::kBF16>(sa, ka[s], qb[s][0], qb[s][1]);
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) r[i] = sa[i] + sb[i];
+  };
+
   for (int si = 0; si < nu; ++si) {
     const int u = u0 + si;
     const int grp = u % p.n_groups, h = (u / p.n_groups) % p.Hkv, b = u / (p.n_groups * p.Hkv);
@@ -945,8 +1073,13 @@ __global__ void __launch_bounds__(Shape<FMT, D>::NW * 32, 1)
     }
     if (si > 0) load_q(u);
 
+    // Online softmax state of this thread's heads 2tig, 2tig+1 (log2 domain).
+    // n = kPLog2 - m; it starts huge but finite, so the first page with a
+    // cached token moves m, and masked scores (-inf) give e = -inf, not NaN.
     float m0 = -kInf, m1 = -kInf, l0 = 0.f, l1 = 0.f;
-    float n0 = kInf, n1 = kInf;  // kPLog2 - m
+    float n0 = 1e30f, n1 = 1e30f;
+    // FP8 attention: running reference max mq and normaliser lq of head gid
+    float mq = -kInf, lq = 0.f;
     float o[MT][4];
 #pragma unroll
     for (int jj = 0; jj < MT; ++jj) o[jj][0] = o[jj][1] = o[jj][2] = o[jj][3] = 0.f;
@@ -957,86 +1090,68 @@ __global__ void __launch_bounds__(Shape<FMT, D>::NW * 32, 1)
     // window mode: tokens of the window's first page before its start are
     // masked (only the unit's relative page 0 can hold such tokens)
     const int n_skip = (p.window > 0 && len > p.window) ? len - p.window - first * kPage : 0;
-    for (int k = warp + j * NW; k < k_end; k += NW, ++j) {
-      const uint8_t* sp = ring + st * F::STAGE;
-      // all lanes agree on the outcome so the warp stays converged
-      if (!__all_sync(0xffffffffu, mbar_wait_bounded(&bars[st], ph))) {
-        if (lane == 0) set_err(p.d_err, kErrTimeout);
-        for (int i = j + 1; i < j + NSW && i < n_local; ++i)  // drain copies in flight
-          mbar_wait_bounded(&bars[i % NSW], (i / NSW) & 1);
-        j = n_local;
-        break;
-      }
-      const bool valid = (stage_ok >> st) & 1u;
 
-      // The stage's words go to registers first, so the stage is refilled with
-      // local item j + NSW before any decode or math on this one (for BF16
-      // head_dim 128, after the QK product: see kLateV).
-      typename F::Raw raw;
-      uint32_t ka[KS][4], va[MT][4];
-      float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
-      // ---- S^T = K Q^T on tensor cores (two accumulator chains)
-      auto qk = [&]() {
-        F::conv_k(raw, ka);
+    // Softmax of page k, part 1: mask the raw scores r of the tokens outside
+    // [t_lo, t_hi) of the page and turn them into exponents e = s - m + kPLog2
+    // (s = c_log2 r).  The running max m moves only when a score passes m +
+    // kRescaleGap (one vote, no reduction, on most pages); p = 2^(s - m) then
+    // stays <= 2^kRescaleGap, which keeps P = p 2^kPLog2 inside f16.
+    auto softmax_e = [&](float r[4], int t_lo, int t_hi, float e[4]) {
+      if constexpr (QP) {
+        // FP8 attention: r holds head gid's raw scores of tokens 2tig,
+        // 2tig+1, 2tig+8, 2tig+9.  P is quantized against the page's own
+        // largest score mp, p = 2^(s - mp), P_hat = E4M3(p / prob_scale);
+        // the page then enters the running sums with weight f = 2^(mp - mq).
+        const int t0 = 2 * tig;
+        if (!(t0 >= t_lo && t0 < t_hi)) r[0] = -kInf;
+        if (!(t0 + 1 >= t_lo && t0 + 1 < t_hi)) r[1] = -kInf;
+        if (!(t0 + 8 >= t_lo && t0 + 8 < t_hi)) r[2] = -kInf;
+        if (!(t0 + 9 >= t_lo && t0 + 9 < t_hi)) r[3] = -kInf;
+        float rmax = fmaxf(fmaxf(r[0], r[1]), fmaxf(r[2], r[3]));
+        rmax = fmaxf(rmax, __shfl_xor_sync(0xffffffffu, rmax, 1));
+        rmax = fmaxf(rmax, __shfl_xor_sync(0xffffffffu, rmax, 2));
+        const bool live = rmax != -kInf;  // the page holds an attended token
+        const float mp = live ? rmax * c_log2 : -kInf;
+        // the running reference moves only when a page max passes it by
+        // more than kRescaleGap, so f <= 2^kRescaleGap
+        if (__any_sync(0xffffffffu, mp > mq + kRescaleGap)) {
+          const float mn = fmaxf(mq, mp);
+          const float a = fast_exp2(mq - mn);  // 0 while mq = -inf
+          lq *= a;
+          const float a0 = __shfl_sync(0xffffffffu, a, 8 * tig);  // head 2tig
+          const float a1 = __shfl_sync(0xffffffffu, a, 8 * tig + 4);  // head 2tig+1
 #pragma unroll
-        for (int s = 0; s < KS; ++s) {
-          if (s & 1)
-            mma16816<F::kBF16>(sb, ka[s], qb[s][0], qb[s][1]);
-          else
-            mma16816<F::kBF16>(sa, ka[s], qb[s][0], qb[s][1]);
+          for (int jj = 0; jj < MT; ++jj) {
+            o[jj][0] *= a0;
+            o[jj][1] *= a1;
+            o[jj][2] *= a0;
+            o[jj][3] *= a1;
+          }
+          mq = mn;
         }
-      };
-      if constexpr (F::kLateV) {
-        if (valid) {
-          F::load_raw_k(sp, gid, tig, raw);
-          qk();
-          F::load_raw_v(sp, gid, tig, raw);
-        }
-      } else if (valid) {
-        F::load_raw(sp, gid, tig, raw);
-      }
-      __syncwarp();
-      if (j + NSW < n_local) issue(j + NSW, st);  // item j + NSW reuses stage st
-      if (++st == NSW) {
-        st = 0;
-        ph ^= 1;
-      }
-      if (!valid) continue;
-      if constexpr (!F::kLateV) qk();
-      F::conv_v(raw, va);
-
-      // raw scores r = q . k_code (the scale c_log2 is applied below)
-      float r0 = sa[0] + sb[0], r1 = sa[1] + sb[1], r2 = sa[2] + sb[2], r3 = sa[3] + sb[3];
-      if (k == k_end - 1 && n_last < kPage) {  // last, partial page: mask tokens past the length
-        const int n_valid = n_last;
-        if (gid >= n_valid) r0 = r1 = -kInf;
-        if (gid + 8 >= n_valid) r2 = r3 = -kInf;
-        const uint32_t m01 = (2 * tig < n_valid ? 0x0000FFFFu : 0u) |
-                             (2 * tig + 1 < n_valid ? 0xFFFF0000u : 0u);
-        const uint32_t m23 = (2 * tig + 8 < n_valid ? 0x0000FFFFu : 0u) |
-                             (2 * tig + 9 < n_valid ? 0xFFFF0000u : 0u);
+        const float f = live ? fast_exp2(mp - mq) : 0.f;
+        const float mpc = live ? mp : 0.f;
+        float pp[4];
 #pragma unroll
-        for (int jj = 0; jj < MT; ++jj) {  // unwritten slots may hold NaN codes
-          va[jj][0] &= m01;
-          va[jj][1] &= m01;
-          va[jj][2] &= m23;
-          va[jj][3] &= m23;
-        }
+        for (int i = 0; i < 4; ++i) pp[i] = fast_exp2(fmaf(r[i], c_log2, -mpc));
+        lq = fmaf(f * 4096.f, (pp[0] + pp[1]) + (pp[2] + pp[3]), lq);  // l carries 2^kPLog2
+        // the decision on fp32 p times fp32(1 / prob_scale), round to nearest even
+        const uint32_t lo = f32x2_to_e4m3x2(pp[0] * inv_ps, pp[1] * inv_ps);
+        const uint32_t hi = f32x2_to_e4m3x2(pp[2] * inv_ps, pp[3] * inv_ps);
+        e[0] = __uint_as_float(lo | (hi << 16));  // B operand of PV: tokens 2tig.. of head gid
+        e[1] = __shfl_sync(0xffffffffu, f, 8 * tig);      // weight of head 2tig
+        e[2] = __shfl_sync(0xffffffffu, f, 8 * tig + 4);  // weight of head 2tig+1
+        return;
       }
-      if (n_skip > 0 && ps == 0 && k == k_base) {  // window's first page: tokens before it
-        if (gid < n_skip) r0 = r1 = -kInf;
-        if (gid + 8 < n_skip) r2 = r3 = -kInf;
-      }
-
-      // ---- online softmax (log2 domain); this thread: heads 2tig, 2tig+1.
-      // The running max m moves only when a score passes m + kRescaleGap
-      // (one vote, no reduction, on most pages); p = 2^(s - m) then stays
-      // <= 2^kRescaleGap, which keeps P = p * 2^kPLog2 inside f16.
-      // e = s - m + kPLog2 with s = c_log2 * r: 2^e = p * 2^kPLog2 = P as fed to the MMA
-      float e0 = fmaf(r0, c_log2, n0), e1 = fmaf(r1, c_log2, n1);
-      float e2 = fmaf(r2, c_log2, n0), e3 = fmaf(r3, c_log2, n1);
-      if (__any_sync(0xffffffffu, e0 > kETop || e2 > kETop || e1 > kETop || e3 > kETop)) {
-        const float s0 = r0 * c_log2, s1 = r1 * c_log2, s2 = r2 * c_log2, s3 = r3 * c_log2;
+      if (!(gid >= t_lo && gid < t_hi)) r[0] = r[1] = -kInf;
+      if (!(gid + 8 >= t_lo && gid + 8 < t_hi)) r[2] = r[3] = -kInf;
+      e[0] = fmaf(r[0], c_log2, n0);
+      e[1] = fmaf(r[1], c_log2, n1);
+      e[2] = fmaf(r[2], c_log2, n0);
+      e[3] = fmaf(r[3], c_log2, n1);
+      if (__any_sync(0xffffffffu, e[0] > kETop || e[2] > kETop || e[1] > kETop || e[3] > kETop)) {
+        const float s0 = r[0] * c_log2, s1 = r[1] * c_log2, s2 = r[2] * c_log2,
+                    s3 = r[3] * c_log2;
         float mx0 = fmaxf(s0, s2), mx1 = fmaxf(s1, s3);
 #pragma unroll
         for (int off = 4; off < 32; off <<= 1) {
@@ -1058,16 +1173,78 @@ __global__ void __launch_bounds__(Shape<FMT, D>::NW * 32, 1)
         m1 = mn1;
         n0 = kPLog2 - m0;
         n1 = kPLog2 - m1;
-        e0 = s0 + n0;
-        e1 = s1 + n1;
-        e2 = s2 + n0;
-        e3 = s3 + n1;
+        e[0] = s0 + n0;
+        e[1] = s1 + n1;
+        e[2] = s2 + n0;
+        e[3] = s3 + n1;
       }
-      const float q0 = fast_exp2(e0), q1 = fast_exp2(e1), q2 = fast_exp2(e2), q3 = fast_exp2(e3);
+    };
+    // Softmax of a page, part 2, and O^T += V^T P^T with the page's V read from
+    // stage stg.  Tokens at or past n_valid are zeroed in V (only the unit's
+    // last page can hold unwritten slots, possibly NaN codes).
+    auto pv_page = [&](const float e[4], int stg, int n_valid) {
+      if constexpr (QP) {
+        // FP8 attention: O^T += f * (V^T P_hat^T) on E4M3 tensor cores.  The A
+        // operand holds, per head-dim row, the codes of tokens 2tig, 2tig+1,
+        // 2tig+8, 2tig+9 (the token order of P_hat): a byte transpose of the
+        // thread's four token rows.
+        typename F::Raw raw;
+        F::load_raw_v(ring + stg * F::STAGE, gid, tig, raw);
+        constexpr int NWD = D / 32;  // 32-bit words of a thread's run of one token row
+        uint32_t x[4][NWD];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const uint32_t* w = reinterpret_cast<const uint32_t*>(&raw.v[i]);
+#pragma unroll
+          for (int k = 0; k < NWD; ++k) x[i][k] = w[k];
+        }
+        uint32_t msk = 0xFFFFFFFFu;
+        if (n_valid < kPage)  // unwritten slots may hold NaN codes
+          msk = (2 * tig < n_valid ? 0x000000FFu : 0u) | (2 * tig + 1 < n_valid ? 0x0000FF00u : 0u) |
+                (2 * tig + 8 < n_valid ? 0x00FF0000u : 0u) |
+                (2 * tig + 9 < n_valid ? 0xFF000000u : 0u);
+        const uint32_t pq = __float_as_uint(e[0]);
+#pragma unroll
+        for (int k = 0; k < NWD; ++k) {
+          const uint32_t xyl = prmt(x[0][k], x[1][k], 0x5140), ztl = prmt(x[2][k], x[3][k], 0x5140);
+          const uint32_t xyh = prmt(x[0][k], x[1][k], 0x7362), zth = prmt(x[2][k], x[3][k], 0x7362);
+          const uint32_t a[4] = {prmt(xyl, ztl, 0x5410) & msk, prmt(xyl, ztl, 0x7632) & msk,
+                                 prmt(xyh, zth, 0x5410) & msk, prmt(xyh, zth, 0x7632) & msk};
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {  // m-tile 2k + hh: head-dim bytes 2hh, 2hh+1 of word k
+            const int jj = 2 * k + hh;
+            float acc[4];
+            mma_e4m3_k16(acc, a[2 * hh], a[2 * hh + 1], pq);
+            o[jj][0] = fmaf(e[1], acc[0], o[jj][0]);
+            o[jj][1] = fmaf(e[2], acc[1], o[jj][1]);
+            o[jj][2] = fmaf(e[1], acc[2], o[jj][2]);
+            o[jj][3] = fmaf(e[2], acc[3], o[jj][3]);
+          }
+        }
+        return;
+      }
+      const float q0 = fast_exp2(e[0]), q1 = fast_exp2(e[1]), q2 = fast_exp2(e[2]),
+                  q3 = fast_exp2(e[3]);
       l0 += q0 + q2;  // l and O carry the factor 2^kPLog2, removed at normalisation
       l1 += q1 + q3;
-
-      // ---- P^T fragments: high part + residual, transposed in registers
+      typename F::Raw raw;
+      uint32_t va[MT][4];
+      F::load_raw_v(ring + stg * F::STAGE, gid, tig, raw);
+      F::conv_v(raw, va);
+      if (n_valid < kPage) {
+        const uint32_t m01 = (2 * tig < n_valid ? 0x0000FFFFu : 0u) |
+                             (2 * tig + 1 < n_valid ? 0xFFFF0000u : 0u);
+        const uint32_t m23 = (2 * tig + 8 < n_valid ? 0x0000FFFFu : 0u) |
+                             (2 * tig + 9 < n_valid ? 0xFFFF0000u : 0u);
+#pragma unroll
+        for (int jj = 0; jj < MT; ++jj) {
+          va[jj][0] &= m01;
+          va[jj][1] &= m01;
+          va[jj][2] &= m23;
+          va[jj][3] &= m23;
+        }
+      }
+      // P^T fragments: high part + residual, transposed in registers
       uint32_t x0h, x1h, x0l, x1l;
       float h0, h1, h2, h3;  // the high parts as fp32
       if constexpr (F::kBF16) {
@@ -1087,28 +1264,76 @@ __global__ void __launch_bounds__(Shape<FMT, D>::NW * 32, 1)
       }
       const uint32_t bh0 = movmatrix_t(x0h), bh1 = movmatrix_t(x1h);
       const uint32_t bl0 = movmatrix_t(x0l), bl1 = movmatrix_t(x1l);
-
-      // ---- O^T += V^T P^T
 #pragma unroll
       for (int jj = 0; jj < MT; ++jj) {
         mma16816<F::kBF16>(o[jj], va[jj], bh0, bh1);
         mma16816<F::kBF16>(o[jj], va[jj], bl0, bl1);
       }
+    };
+    // Valid token range [t_lo, t_hi) of page k (before the last-page cut).
+    auto t_lo_of = [&](int k, bool valid) {
+      return !valid ? kPage : (n_skip > 0 && ps == 0 && k == k_base) ? n_skip : 0;
+    };
+
+    // Software pipeline over this warp's pages of the segment: while page C's
+    // softmax and PV run, page N's K is read and its QK issued, two
+    // independent dependency chains in one straight-line block.
+    int kc = warp + j * NW;  // this warp's first page of the segment
+    if (!dead && kc < k_end && wait_item()) {
+      float rc[4];
+      bool vc = (stage_ok >> st) & 1u;
+      int stc = st;
+      qk_page(stc, rc);
+      advance();
+      for (int kn = kc + NW; kn < k_end; kn += NW) {
+        float ec[4];
+        softmax_e(rc, t_lo_of(kc, vc), kPage, ec);  // C is not the segment's last page
+        if (!wait_item()) break;
+        const bool vn = (stage_ok >> st) & 1u;
+        const int stn = st;
+        float rn[4];
+        qk_page(stn, rn);        // chain 1: page N
+        pv_page(ec, stc, kPage);  // chain 2: page C
+        refill(stc);
+        advance();
+        kc = kn;
+        stc = stn;
+        vc = vn;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) rc[i] = rn[i];
+      }
+      if (!dead) {  // the warp's last page of the segment
+        const int t_hi = (kc == k_end - 1 && n_last < kPage) ? n_last : kPage;
+        float ec[4];
+        softmax_e(rc, t_lo_of(kc, vc), t_hi, ec);
+        pv_page(ec, stc, t_hi);
+        refill(stc);
+      }
     }
+    if (dead) j = n_local;  // no further segment reads a page
     k_base = k_end;
 
-#pragma unroll
-    for (int off = 4; off < 32; off <<= 1) {
-      l0 += __shfl_xor_sync(0xffffffffu, l0, off);
-      l1 += __shfl_xor_sync(0xffffffffu, l1, off);
-    }
     // ---- segment end: warp partials -> shared slots, merged by the CTA
     float* wp = slots + warp * S::WPART;  // m[8], l[8], o[8][D]
-    if (gid == 0) {
-      wp[2 * tig] = m0;
-      wp[2 * tig + 1] = m1;
-      wp[8 + 2 * tig] = l0;
-      wp[8 + 2 * tig + 1] = l1;
+    if constexpr (QP) {  // head gid's sums are spread over the tig lanes
+      lq += __shfl_xor_sync(0xffffffffu, lq, 1);
+      lq += __shfl_xor_sync(0xffffffffu, lq, 2);
+      if (tig == 0) {
+        wp[gid] = mq;
+        wp[8 + gid] = lq;
+      }
+    } else {
+#pragma unroll
+      for (int off = 4; off < 32; off <<= 1) {
+        l0 += __shfl_xor_sync(0xffffffffu, l0, off);
+        l1 += __shfl_xor_sync(0xffffffffu, l1, off);
+      }
+      if (gid == 0) {
+        wp[2 * tig] = m0;
+        wp[2 * tig + 1] = m1;
+        wp[8 + 2 * tig] = l0;
+        wp[8 + 2 * tig + 1] = l1;
+      }
     }
 #pragma unroll
     for (int jj = 0; jj < MT; ++jj) {
@@ -1148,7 +1373,7 @@ __global__ void __launch_bounds__(Shape<FMT, D>::NW * 32, 1)
         const int qi = grp * 8 + hh;
         if (qi < p.G) {
           const size_t row = static_cast<size_t>(b) * p.Hq + h * p.G + qi;
-          p.out[row * D + d] = L > 0.f ? acc * (vs / L) : 0.f;
+          p.out[row * D + d] = L > 0.f ? acc * (vs_out / L) : 0.f;
           if (d == 0 && p.lse) p.lse[row] = L > 0.f ? (M + log2f(L) - kPLog2) * kLn2 : -kInf;
         }
       } else {
@@ -1171,7 +1396,7 @@ __global__ void __launch_bounds__(Shape<FMT, D>::NW * 32, 1)
       }
       __syncthreads();
       if (s_last) {
-        final_merge<D, S::WPART>(p, u, b, h, grp, c_first, c_last - c_first + 1, vs, tid, NT);
+        final_merge<D, S::WPART>(p, u, b, h, grp, c_first, c_last - c_first + 1, vs_out, tid, NT);
         if (tid == 0) p.ws_cnt[u] = 0u;  // ready for the next launch
       }
     }
@@ -1186,13 +1411,13 @@ size_t smem_bytes() {
          sizeof(float) * S::NW * S::WPART + 8 * static_cast<size_t>(S::NW) * S::NSW;
 }
 
-template <int FMT, int D>
+template <int FMT, int D, bool QP = false>
 cudaError_t launch_t(const CUtensorMap* maps, const DecodeParams& p, int ctas,
                      cudaStream_t stream) {
   using S = Shape<FMT, D>;
   const size_t smem = smem_bytes<FMT, D>();
-  static std::atomic<bool> attr_done[kMaxDevices];  // per device ordinal
-  cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kvq_decode_kernel<FMT, D>),
+  static std::atomic<bool> attr_done[kMaxDevices];  // per instantiation and device ordinal
+  cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kvq_decode_kernel<FMT, D, QP>),
                                    smem, attr_done);
   if (e != cudaSuccess) return e;
   // Programmatic stream serialization: the launch may begin while a
@@ -1207,7 +1432,8 @@ cudaError_t launch_t(const CUtensorMap* maps, const DecodeParams& p, int ctas,
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kvq_decode_kernel<FMT, D>, maps[0], maps[1], maps[2], maps[3], p);
+  return cudaLaunchKernelEx(&cfg, kvq_decode_kernel<FMT, D, QP>, maps[0], maps[1], maps[2], maps[3],
+                            p);
 }
 
 template <int FMT, int D>
@@ -1234,7 +1460,12 @@ bool decode_config(int fmt, int D, DecodeConfig* cfg) {
 }
 
 cudaError_t launch_decode(int fmt, int D, const CUtensorMap* maps, const DecodeParams& p,
-                          int ctas, cudaStream_t stream) {
+                          int ctas, cudaStream_t stream, bool fp8_qp) {
+  if (fp8_qp) {
+    if (fmt != 1) return cudaErrorInvalidValue;
+    return D == 128 ? launch_t<1, 128, true>(maps, p, ctas, stream)
+                    : launch_t<1, 64, true>(maps, p, ctas, stream);
+  }
   switch (fmt * 1000 + D) {
     case 64: return launch_t<0, 64>(maps, p, ctas, stream);
     case 128: return launch_t<0, 128>(maps, p, ctas, stream);

@@ -147,6 +147,29 @@ __device__ __forceinline__ void mma_bf16(float c[4], const uint32_t a[4], uint32
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+// D = A * B + C, m16n8k32 with E4M3 operands, fp32 accumulate.  A row-major
+// 16x32 (four registers of four codes: rows g / g+8, k 4t..4t+3 / 16+4t..),
+// B 32x8 (two registers: k 4t..4t+3 / 16+4t.., column g).
+__device__ __forceinline__ void mma_e4m3_k32(float c[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                             uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.f32.e4m3.e4m3.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};\n"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+// D = A * B, m16n8k16 with E4M3 operands, fp32 result.  A 16x16 (two
+// registers: rows g / g+8, k 4t..4t+3), B 16x8 (one register: k 4t..4t+3,
+// column g).
+__device__ __forceinline__ void mma_e4m3_k16(float d[4], uint32_t a0, uint32_t a1, uint32_t b0) {
+  const float z = 0.f;
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.e4m3.e4m3.f32 {%0,%1,%2,%3}, {%4,%5}, {%6}, "
+      "{%7,%7,%7,%7};\n"
+      : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+      : "r"(a0), "r"(a1), "r"(b0), "f"(z));
+}
+
 // Transpose of an 8x8 16-bit matrix held in the mma accumulator layout.
 __device__ __forceinline__ uint32_t movmatrix_t(uint32_t x) {
   uint32_t r;

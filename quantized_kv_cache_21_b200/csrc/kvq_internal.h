@@ -17,6 +17,8 @@ struct DecodeParams {
   const int32_t* seq_lens;    // [B]
   const float* k_scale;       // device scalar (FP8: s, NVFP4: g); unused for BF16
   const float* v_scale;
+  const float* q_scale;       // FP8 attention only: device scalar, E4M3 scale of q
+  const float* prob_scale;    // FP8 attention only: device scalar, E4M3 scale of P
   float* out;                 // [B][Hq][D]
   float* lse;                 // [B][Hq] or null
   float* ws_part;             // [units + ctas][16 + 8 D] per-CTA partials (slot u + cta)
@@ -42,9 +44,10 @@ struct DecodeConfig {
 
 // Per-(format, head_dim) kernel configuration; false if unsupported.
 bool decode_config(int fmt, int D, DecodeConfig* cfg);
-// Launch the decode kernel on `ctas` persistent CTAs.
+// Launch the decode kernel on `ctas` persistent CTAs.  fp8_qp: the FP8
+// attention variant (FP8 cache only; E4M3 Q and P on E4M3 tensor-core MMAs).
 cudaError_t launch_decode(int fmt, int D, const CUtensorMap* maps, const DecodeParams& p,
-                          int ctas, cudaStream_t stream);
+                          int ctas, cudaStream_t stream, bool fp8_qp = false);
 
 struct PrefillParams {
   const uint16_t* q;          // [B][Tq][Hq][D] bf16: the Tq newest tokens of each sequence

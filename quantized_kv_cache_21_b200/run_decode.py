@@ -6,7 +6,8 @@
 Builds the named workload's cache (optionally with another format, context
 length, batch or head_dim), writes the step's tokens with kv_quantize_write,
 then launches kv_decode_attention (with --prefill: kv_prefill_attention of the
-step's chunk of new tokens) --launches times on the current stream and prints
+step's chunk of new tokens; with --fp8qp: kv_decode_attention_fp8qp over the
+FP8 cache) --launches times on the current stream and prints
 the device error word and the KV-scan bytes (prefill: algorithmic FLOPs) of one
 launch.  Nothing is timed here: bench.py owns timing."""
 from __future__ import annotations
@@ -30,6 +31,8 @@ def main(argv=None) -> int:
     ap.add_argument("--launches", type=int, default=4)
     ap.add_argument("--prefill", action="store_true",
                     help="launch the chunk's prefill attention instead of the decode")
+    ap.add_argument("--fp8qp", action="store_true",
+                    help="launch the FP8 attention (E4M3 q and P) over an FP8 cache")
     args = ap.parse_args(argv)
     w = wl.WORKLOADS[args.workload]
     over = {}
@@ -44,8 +47,15 @@ def main(argv=None) -> int:
     sc.write()  # the step's own tokens, so the scanned cache is complete
     if args.prefill:
         sc.prefill_setup()
+    if args.fp8qp:
+        sc.fp8qp_setup()
     for _ in range(args.launches):
-        sc.prefill() if args.prefill else sc.decode()
+        if args.prefill:
+            sc.prefill()
+        elif args.fp8qp:
+            sc.decode_fp8qp()
+        else:
+            sc.decode()
     torch.cuda.synchronize()
     what = (f"prefill chunk {sc.chunk}, FLOPs per launch {sc.prefill_flops}" if args.prefill
             else f"KV-scan bytes per launch {sc.scan_bytes}")

@@ -160,6 +160,28 @@ class DecodeScenario:
     def window_scan_bytes(self, window: int) -> int:
         return kv_scan_bytes(self.fmt, np.minimum(self.lens, window), self.H, self.D)
 
+    # ---- FP8 attention (E4M3 q and P) over the FP8 cache
+    def fp8qp_setup(self):
+        """Per-layer E4M3 scales of q (calibrated on the step's query with the
+        library's abs-max and scale kernels) and of P (the same formula at an
+        observed maximum of 1)."""
+        if hasattr(self, "d_qs"):
+            return
+        assert self.fmt == "fp8", "FP8 attention runs on the FP8 cache"
+        amax = torch.zeros(1, dtype=torch.float32, device=self.device)
+        kvq.kv_calibrate_absmax(self.q.contiguous(), amax)
+        self.d_qs = torch.empty(1, dtype=torch.float32, device=self.device)
+        kvq.kv_scale_from_absmax_device("fp8", amax, self.d_qs)
+        self.d_ps = torch.tensor([kvq.kv_scale_from_absmax("fp8", 1.0)], dtype=torch.float32,
+                                 device=self.device)
+
+    def decode_fp8qp(self, stream=None, out=None, lse=None):
+        kvq.kv_decode_attention_fp8qp(self.q, self.cache, self.d_bt, self.d_lens, self.L,
+                                      self.d_ks, self.d_vs, self.d_qs, self.d_ps,
+                                      self.out if out is None else out,
+                                      self.lse if lse is None else lse, self.ws, self.err,
+                                      stream=stream)
+
     def step(self, stream=None):
         self.write(stream)
         self.decode(stream)
