@@ -29,7 +29,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "kvq_oracle.c")
 _LIB = os.path.join(_HERE, "libkvq_oracle.so")
 
-FORMATS = {"bf16": 0, "fp8": 1, "nvfp4": 2}
+FORMATS = {"bf16": 0, "fp8": 1, "nvfp4": 2, "pq3": 3, "f32": 4}
 PAGE = 16
 
 
@@ -96,6 +96,18 @@ def lib():
         L.orc_prefill_attention.argtypes = [i32, P, P, P, i64, i32, i32, P, i32, P, i32, i32,
                                             i32, f32, f32, f64, P, i64, P, P]
         L.orc_merge.argtypes = [i32, i32, P, P, P, P, P]
+        L.orc_lloyd_max_gaussian.restype = None
+        L.orc_lloyd_max_gaussian.argtypes = [i32, P]
+        L.orc_pq3_codebook.restype = None
+        L.orc_pq3_codebook.argtypes = [P]
+        L.orc_pq3_encode_row.restype = None
+        L.orc_pq3_encode_row.argtypes = [P, P, P, P]
+        L.orc_pq3_decode_row.restype = None
+        L.orc_pq3_decode_row.argtypes = [f32, P, P, P]
+        L.orc_pq3_write.restype = i32
+        L.orc_pq3_write.argtypes = [P, P, i64, i32, P, i64, P, P, P, P]
+        L.orc_pq3_to_f32.restype = None
+        L.orc_pq3_to_f32.argtypes = [P, P, i64, i32, P, P, P, P]
         L.orc_decode_attention_fp8qp.restype = i32
         L.orc_decode_attention_fp8qp.argtypes = [P, P, P, i64, i32, i32, P, i32, P, i32, i32,
                                                  f32, f32, f32, f32, f64, f64, P, i64, P, P, P]
@@ -333,3 +345,82 @@ def decode_attention_fp8qp(q_bits, k_cache, v_cache, H: int, block_table, seq_le
     if rc:
         raise ValueError(f"oracle fp8 q/p attention failed ({rc})")
     return out, lse, amb
+
+
+# --------------------------------------------------------------------------- PQ3 codec
+# The 3-bit planar-rotation codec of 128-element vectors ("AMD MI300X - KV
+# Cache Compression Benchmark", "Key Results": 52-byte blocks, 4.923x against
+# FP16); see kvq_oracle.c for the reading the oracle takes.
+PQ3_D = 128
+PQ3_PARAMS = 136  # 8 codebook values + 64 (cos, sin) pairs
+
+
+def lloyd_max_gaussian(n: int) -> np.ndarray:
+    """Centroids of the n-level Lloyd-Max quantizer of N(0, 1) (float64)."""
+    c = np.empty(n, np.float64)
+    lib().orc_lloyd_max_gaussian(n, _p(c))
+    return c
+
+
+def pq3_codebook() -> np.ndarray:
+    cb = np.empty(8, np.float32)
+    lib().orc_pq3_codebook(_p(cb))
+    return cb
+
+
+def pq3_params(cos_sin) -> np.ndarray:
+    """The parameter block of one tensor: the codebook, then the 64 given
+    (cos, sin) pairs (fp32)."""
+    cs = _c(cos_sin, np.float32).reshape(64, 2)
+    return np.concatenate([pq3_codebook(), cs.reshape(-1)]).astype(np.float32)
+
+
+def pq3_encode_row(x_bits, params):
+    """(norm, indices[128]) of one 128-element BF16 row."""
+    x = _c(x_bits, np.uint16).reshape(PQ3_D)
+    pr = _c(params, np.float32)
+    nrm = np.empty(1, np.float32)
+    idx = np.empty(PQ3_D, np.uint8)
+    lib().orc_pq3_encode_row(_p(x), _p(pr), _p(nrm), _p(idx))
+    return float(nrm[0]), idx
+
+
+def pq3_decode_row(nrm, idx, params) -> np.ndarray:
+    i = _c(idx, np.uint8).reshape(PQ3_D)
+    pr = _c(params, np.float32)
+    out = np.empty(PQ3_D, np.float32)
+    lib().orc_pq3_decode_row(float(np.float32(nrm)), _p(i), _p(pr), _p(out))
+    return out
+
+
+def pq3_write(k_bits, v_bits, slot_mapping, k_cache, v_cache, k_params, v_params) -> int:
+    """Quantize-on-write of BF16 K/V rows ([T][H][128]) into PQ3 caches (byte
+    buffers of num_blocks * H * 832 bytes) at the given physical slots."""
+    k = _c(k_bits, np.uint16)
+    v = _c(v_bits, np.uint16)
+    T, H, D = k.shape
+    assert D == PQ3_D
+    sm = _c(slot_mapping, np.int64)
+    nb = k_cache.size // (H * head_page_bytes("pq3", D))
+    kp, vp = _c(k_params, np.float32), _c(v_params, np.float32)
+    return int(lib().orc_pq3_write(_p(k), _p(v), T, H, _p(sm), nb, _p(k_cache), _p(v_cache),
+                                   _p(kp), _p(vp)))
+
+
+def pq3_to_f32(k_cache, v_cache, H: int, k_params, v_params):
+    """The dequantised caches in the "f32" format ([blocks][H][16][128] fp32,
+    as byte buffers) the attention oracle reads."""
+    nb = k_cache.size // (H * head_page_bytes("pq3", PQ3_D))
+    ko = np.empty(nb * H * PAGE * PQ3_D, np.float32)
+    vo = np.empty(nb * H * PAGE * PQ3_D, np.float32)
+    kp, vp = _c(k_params, np.float32), _c(v_params, np.float32)
+    lib().orc_pq3_to_f32(_p(k_cache), _p(v_cache), nb, H, _p(kp), _p(vp), _p(ko), _p(vo))
+    return ko.view(np.uint8), vo.view(np.uint8)
+
+
+def pq3_decode_attention(q_bits, k_cache, v_cache, H: int, block_table, seq_lens, k_params,
+                         v_params, sm_scale=None, pairs=None, window=0):
+    """Float64 decode attention over the dequantised PQ3 cache."""
+    kf, vf = pq3_to_f32(k_cache, v_cache, H, k_params, v_params)
+    return decode_attention("f32", q_bits, kf, vf, H, block_table, seq_lens, 1.0, 1.0,
+                            sm_scale=sm_scale, pairs=pairs, window=window)

@@ -44,6 +44,7 @@
 #define ORC_BF16 0
 #define ORC_FP8 1
 #define ORC_NVFP4 2
+#define ORC_F32 4 /* plain fp32 values, the dequantised form of another format */
 
 #define ORC_PAGE 16 /* tokens per cache page (block size) */
 
@@ -240,7 +241,9 @@ static int64_t head_page_index(int64_t blk, int h, int H) { return blk * H + h; 
 static float dequant_elem(int fmt, const void* cache, int64_t blk, int h, int o, int d, int H,
                           int D, float scale) {
   int64_t hp = head_page_index(blk, h, H);
-  if (fmt == ORC_BF16) {
+  if (fmt == ORC_F32) {
+    return ((const float*)cache)[(hp * ORC_PAGE + o) * D + d];
+  } else if (fmt == ORC_BF16) {
     const uint16_t* c = (const uint16_t*)cache;
     return bf16_to_f32(c[(hp * ORC_PAGE + o) * D + d]);
   } else if (fmt == ORC_FP8) {
@@ -257,6 +260,8 @@ static float dequant_elem(int fmt, const void* cache, int64_t blk, int h, int o,
 }
 
 int64_t orc_head_page_bytes(int fmt, int D) {
+  if (fmt == ORC_F32) return (int64_t)ORC_PAGE * D * 4;
+  if (fmt == 3) return (int64_t)ORC_PAGE * 52; /* PQ3, D = 128 (see below) */
   if (fmt == ORC_BF16) return (int64_t)ORC_PAGE * D * 2;
   if (fmt == ORC_FP8) return (int64_t)ORC_PAGE * D;
   return (int64_t)9 * D;
@@ -697,4 +702,207 @@ int orc_decode_attention_fp8qp(const uint16_t* q, const uint8_t* k_cache, const 
     free(w);
   }
   return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* PQ3: 3-bit planar-rotation codec of 128-element vectors (52-byte blocks)  */
+/* ------------------------------------------------------------------------ */
+/*
+ * [MI300X] "AMD MI300X - KV Cache Compression Benchmark", "Key Results": the
+ * 3-bit methods share one 52-byte block layout at 4.923x compression against
+ * FP16 (a 128-element FP16 vector is 256 bytes; 256 / 52 = 4.923), with a
+ * reconstruction cosine similarity of 0.983; PlanarQuant needs the fewest
+ * FMAs (256 against 16,384 for a dense 128 x 128 rotation), and the
+ * repository lists a Lloyd-Max solver and codebook generator.  The page fixes
+ * no more; the plain reading this oracle takes:
+ *   block  = one 128-element head vector: its fp32 L2 norm (4 bytes) and 128
+ *            3-bit codebook indices (48 bytes);
+ *   rotate = 64 planar rotations of the coordinate pairs (2j, 2j+1) by
+ *            seeded angles, given as fp32 (cos_j, sin_j) (4 multiplies a
+ *            pair: the 256 FMAs);
+ *   codebook = the 8-level Lloyd-Max quantizer of N(0, 1/128), the law of
+ *            one coordinate of a random unit vector in 128 dimensions
+ *            (Gaussian approximation), rounded to f16 values;
+ *   encode = u = x / |x|, y = R u, index = nearest codebook value;
+ *   decode = |x| * R^T c[index].
+ * Every fp32 step of the encode is fixed so the indices are exact:
+ *   ss  = sum of x_i^2 as a pairwise tree in index order (level 1 adds
+ *         elements 2i and 2i+1, each further level adds adjacent sums);
+ *   nrm = sqrt(ss) rounded to nearest; u_i = x_i / nrm (IEEE division);
+ *   y_2j = fmaf(c_j, u_2j, -(s_j * u_2j+1)), y_2j+1 = fmaf(s_j, u_2j, c_j * u_2j+1);
+ *   index = number of thresholds t_k = (c_k + c_k+1) / 2 (fp32) below y
+ *         (y equal to a threshold takes the lower index);
+ *   nrm = 0 (an all-zero vector) stores norm 0 and indices 0.
+ * The dequantised element (fp32): with Y0 = c[i_2j], Y1 = c[i_2j+1],
+ *   x_hat_2j = nrm * fmaf(c_j, Y0, s_j * Y1), x_hat_2j+1 = nrm * fmaf(c_j, Y1, -(s_j * Y0)).
+ * Layout of a 16-token head page (832 bytes): the 16 norms (fp32), then 16
+ * rows of 48 index bytes; index i of a row sits in bits [3i, 3i+3) of the
+ * row's little-endian bit string.
+ * The per-layer parameter block of a tensor (K or V): 8 codebook values then
+ * the 64 (cos, sin) pairs, 136 fp32.
+ */
+#define ORC_PQ3 3
+#define ORC_PQ3_D 128
+#define ORC_PQ3_PAGE_BYTES (ORC_PAGE * 4 + ORC_PAGE * 48)
+
+/* Standard normal density and distribution function. */
+static double std_pdf(double x) { return exp(-0.5 * x * x) / sqrt(2.0 * 3.14159265358979323846); }
+static double std_cdf(double x) { return 0.5 * erfc(-x / sqrt(2.0)); }
+
+/* The n-level Lloyd-Max quantizer of N(0, 1): centroids c_0 < ... < c_{n-1}
+ * satisfying both conditions (each threshold is the midpoint of its two
+ * centroids; each centroid is the mean of the density over its cell),
+ * reached by Lloyd's fixed-point iteration from equally spaced centroids. */
+void orc_lloyd_max_gaussian(int n, double* c) {
+  for (int k = 0; k < n; k++) c[k] = -2.0 + 4.0 * (k + 0.5) / n;
+  for (int it = 0; it < 100000; it++) {
+    double change = 0.0;
+    for (int k = 0; k < n; k++) {
+      double lo = k == 0 ? -INFINITY : 0.5 * (c[k - 1] + c[k]);
+      double hi = k == n - 1 ? INFINITY : 0.5 * (c[k] + c[k + 1]);
+      double mass = std_cdf(hi) - std_cdf(lo);
+      double mean = (std_pdf(lo) - std_pdf(hi)) / mass; /* E[X | lo < X < hi] */
+      change = fmax(change, fabs(mean - c[k]));
+      c[k] = mean;
+    }
+    if (change < 1e-15) break;
+  }
+}
+
+/* Round a double to the nearest f16 value (ties to even), as a double; the
+ * values here are normal f16 numbers (|v| in [2^-14, 65504]). */
+static double round_to_f16(double v) {
+  int e;
+  frexp(v, &e);                   /* v = f * 2^e, f in [0.5, 1) */
+  double ulp = ldexp(1.0, e - 11); /* 11 significant bits */
+  return round_half_even(fabs(v) / ulp) * ulp * (v < 0 ? -1.0 : 1.0);
+}
+
+/* The PQ3 codebook: the 8-level Lloyd-Max centroids scaled by 1/sqrt(128),
+ * rounded to f16, as fp32. */
+void orc_pq3_codebook(float* cb) {
+  double c[8];
+  orc_lloyd_max_gaussian(8, c);
+  for (int k = 0; k < 8; k++) cb[k] = (float)round_to_f16(c[k] / sqrt(128.0));
+}
+
+/* Pairwise-tree fp32 sum of squares of a 128-element BF16 row. */
+static float pq3_sum_squares(const uint16_t* x) {
+  float s[ORC_PQ3_D];
+  for (int i = 0; i < ORC_PQ3_D; i++) {
+    float v = bf16_to_f32(x[i]);
+    s[i] = v * v; /* exact: a BF16 square has at most 16 significant bits */
+  }
+  for (int n = ORC_PQ3_D; n > 1; n /= 2)
+    for (int i = 0; i < n / 2; i++) s[i] = s[2 * i] + s[2 * i + 1];
+  return s[0];
+}
+
+/* Encode one row: norm and 128 indices (one byte each here). */
+static void pq3_encode(const uint16_t* x, const float* params, float* nrm_out, uint8_t* idx) {
+  const float* cb = params;
+  const float* rot = params + 8;
+  float nrm = sqrtf(pq3_sum_squares(x));
+  *nrm_out = nrm;
+  if (nrm == 0.0f) {
+    for (int i = 0; i < ORC_PQ3_D; i++) idx[i] = 0;
+    return;
+  }
+  float thr[7];
+  for (int k = 0; k < 7; k++) thr[k] = (cb[k] + cb[k + 1]) / 2.0f;
+  for (int j = 0; j < ORC_PQ3_D / 2; j++) {
+    float c = rot[2 * j], s = rot[2 * j + 1];
+    float u0 = bf16_to_f32(x[2 * j]) / nrm, u1 = bf16_to_f32(x[2 * j + 1]) / nrm;
+    float y[2];
+    y[0] = fmaf(c, u0, -(s * u1));
+    y[1] = fmaf(s, u0, c * u1);
+    for (int h = 0; h < 2; h++) {
+      int k = 0;
+      while (k < 7 && y[h] > thr[k]) k++;
+      idx[2 * j + h] = (uint8_t)k;
+    }
+  }
+}
+
+/* The dequantised fp32 row of a norm and 128 indices. */
+static void pq3_decode(float nrm, const uint8_t* idx, const float* params, float* out) {
+  const float* cb = params;
+  const float* rot = params + 8;
+  for (int j = 0; j < ORC_PQ3_D / 2; j++) {
+    float c = rot[2 * j], s = rot[2 * j + 1];
+    float y0 = cb[idx[2 * j]], y1 = cb[idx[2 * j + 1]];
+    out[2 * j] = nrm * fmaf(c, y0, s * y1);
+    out[2 * j + 1] = nrm * fmaf(c, y1, -(s * y0));
+  }
+}
+
+static void pq3_pack(const uint8_t* idx, uint8_t* bytes48) {
+  for (int b = 0; b < 48; b++) bytes48[b] = 0;
+  for (int i = 0; i < ORC_PQ3_D; i++)
+    for (int k = 0; k < 3; k++)
+      if ((idx[i] >> k) & 1) bytes48[(3 * i + k) / 8] |= (uint8_t)(1u << ((3 * i + k) % 8));
+}
+
+static void pq3_unpack(const uint8_t* bytes48, uint8_t* idx) {
+  for (int i = 0; i < ORC_PQ3_D; i++) {
+    int v = 0;
+    for (int k = 0; k < 3; k++) v |= ((bytes48[(3 * i + k) / 8] >> ((3 * i + k) % 8)) & 1) << k;
+    idx[i] = (uint8_t)v;
+  }
+}
+
+/* Encode / decode one row (exposed for the checks). */
+void orc_pq3_encode_row(const uint16_t* x, const float* params, float* nrm, uint8_t* idx) {
+  pq3_encode(x, params, nrm, idx);
+}
+void orc_pq3_decode_row(float nrm, const uint8_t* idx, const float* params, float* out) {
+  pq3_decode(nrm, idx, params, out);
+}
+
+/* Quantize-on-write of tokens [0, T) of k, v ([T][H][128] BF16) to the
+ * physical slots slot_mapping[t] (negative: skip).  Returns -1 if a slot lies
+ * beyond the cache (nothing written for it), else 0. */
+int orc_pq3_write(const uint16_t* k, const uint16_t* v, int64_t T, int H,
+                  const int64_t* slot_mapping, int64_t num_blocks, uint8_t* k_cache,
+                  uint8_t* v_cache, const float* k_params, const float* v_params) {
+  int rc = 0;
+  for (int64_t t = 0; t < T; t++) {
+    int64_t slot = slot_mapping[t];
+    if (slot < 0) continue;
+    int64_t blk = slot / ORC_PAGE;
+    int o = (int)(slot % ORC_PAGE);
+    if (blk >= num_blocks) {
+      rc = -1;
+      continue;
+    }
+    for (int h = 0; h < H; h++)
+      for (int kv = 0; kv < 2; kv++) {
+        const uint16_t* x = (kv ? v : k) + (t * H + h) * ORC_PQ3_D;
+        uint8_t* page = (kv ? v_cache : k_cache) + (blk * H + h) * (int64_t)ORC_PQ3_PAGE_BYTES;
+        float nrm;
+        uint8_t idx[ORC_PQ3_D];
+        pq3_encode(x, kv ? v_params : k_params, &nrm, idx);
+        memcpy(page + 4 * o, &nrm, 4);
+        pq3_pack(idx, page + ORC_PAGE * 4 + 48 * o);
+      }
+  }
+  return rc;
+}
+
+/* Dequantise the whole PQ3 cache into fp32 caches [num_blocks][H][16][128]
+ * (the float format the attention oracle reads). */
+void orc_pq3_to_f32(const uint8_t* k_cache, const uint8_t* v_cache, int64_t num_blocks, int H,
+                    const float* k_params, const float* v_params, float* k_out, float* v_out) {
+  for (int64_t hp = 0; hp < num_blocks * H; hp++)
+    for (int kv = 0; kv < 2; kv++) {
+      const uint8_t* page = (kv ? v_cache : k_cache) + hp * (int64_t)ORC_PQ3_PAGE_BYTES;
+      float* dst = (kv ? v_out : k_out) + hp * ORC_PAGE * ORC_PQ3_D;
+      for (int o = 0; o < ORC_PAGE; o++) {
+        float nrm;
+        uint8_t idx[ORC_PQ3_D];
+        memcpy(&nrm, page + 4 * o, 4);
+        pq3_unpack(page + ORC_PAGE * 4 + 48 * o, idx);
+        pq3_decode(nrm, idx, kv ? v_params : k_params, dst + o * ORC_PQ3_D);
+      }
+    }
 }

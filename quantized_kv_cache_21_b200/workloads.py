@@ -82,6 +82,14 @@ def physical_slots(block_table: np.ndarray, b: int, positions: np.ndarray) -> np
     return block_table[b, pos // PAGE].astype(np.int64) * PAGE + pos % PAGE
 
 
+def planar_rotation(rng: np.random.Generator, pairs: int = 64) -> np.ndarray:
+    """[pairs][2] fp32 (cos, sin) of seeded angles uniform in [0, 2 pi): the
+    random planar rotation a 3-bit rotation codec applies to each head vector
+    (an input drawn once per tensor, like a scale)."""
+    theta = rng.uniform(0.0, 2.0 * np.pi, size=pairs)
+    return np.stack([np.cos(theta), np.sin(theta)], axis=1).astype(np.float32)
+
+
 def varlen(rng: np.random.Generator, B: int, L: int) -> np.ndarray:
     """Per-sequence lengths uniform in [ceil(L/2), L]."""
     return rng.integers((L + 1) // 2, L + 1, size=B).astype(np.int32)
