@@ -100,6 +100,7 @@ struct Fmt<1, 128> {
   struct Raw {
     uint4 k[4], v[4];
   };
+  static constexpr bool kLateV = false;
   __device__ static void load_raw_k(const uint8_t* st, int gid, int tig, Raw& r) {
 #pragma unroll
     for (int rr = 0; rr < 2; ++rr) {
@@ -160,6 +161,7 @@ struct Fmt<1, 64> {
     uint4 k[2];
     uint2 v[4];
   };
+  static constexpr bool kLateV = false;
   __device__ static void load_raw_k(const uint8_t* st, int gid, int tig, Raw& r) {
 #pragma unroll
     for (int rr = 0; rr < 2; ++rr) r.k[rr] = lds128(st + swz64(gid + 8 * rr, 16 * tig));
@@ -214,6 +216,7 @@ struct Fmt<0, 64> {
   struct Raw {
     uint4 k[4], v[4];
   };
+  static constexpr bool kLateV = false;
   __device__ static void load_raw_k(const uint8_t* st, int gid, int tig, Raw& r) {
 #pragma unroll
     for (int rr = 0; rr < 2; ++rr) {
@@ -284,6 +287,9 @@ struct Fmt<0, 128> {
   struct Raw {
     uint4 k[8], v[8];
   };
+  // 64 raw registers would not fit beside the accumulators: K is read and
+  // used first, V read after the QK product (kLateV), then the stage refilled.
+  static constexpr bool kLateV = true;
   __device__ static void load_raw_k(const uint8_t* st, int gid, int tig, Raw& r) {
 #pragma unroll
     for (int hf = 0; hf < 2; ++hf) {
@@ -379,6 +385,7 @@ struct Fmt<2, 64> {
     uint2 k[2];
     uint32_t v[4], ks[2], vs[4];
   };
+  static constexpr bool kLateV = false;
   __device__ static void load_raw_k(const uint8_t* st, int gid, int tig, Raw& r) {
 #pragma unroll
     for (int rr = 0; rr < 2; ++rr) {
@@ -465,6 +472,7 @@ struct Fmt<2, 128> {
     uint2 v[4];
     uint32_t ks[2], vs[4];
   };
+  static constexpr bool kLateV = false;
   __device__ static void load_raw_k(const uint8_t* st, int gid, int tig, Raw& r) {
 #pragma unroll
     for (int rr = 0; rr < 2; ++rr) {
@@ -919,16 +927,6 @@ __global__ void __launch_bounds__(Shape<FMT, D>::NW * 32, 1)
   // no data.
   unsigned ok_win = __ballot_sync(0xffffffffu, cur_blk >= 0 && cur_blk < p.num_blocks);
   unsigned stage_ok = 0;
-  // A stage whose block id is bad gets no copy: the warp zero-fills it (so no
-  // stale or unwritten bytes, possibly NaN codes, reach the V product) and
-  // completes its phase by hand; the page's scores are masked, so it carries
-  // no weight.
-  auto fill_bad = [&](int stg) {
-    uint4* z = reinterpret_cast<uint4*>(ring + stg * F::STAGE);
-#pragma unroll 1
-    for (int i = lane; i < F::STAGE / 16; i += 32) z[i] = make_uint4(0u, 0u, 0u, 0u);
-    __syncwarp();
-  };
   auto issue = [&](int i, int stg) {
     if (i >= chunk + 32) {  // slide the id window by 32 items
       chunk += 32;
@@ -940,7 +938,6 @@ __global__ void __launch_bounds__(Shape<FMT, D>::NW * 32, 1)
     const int src = i - chunk;
     const unsigned ok = (ok_win >> src) & 1u;
     stage_ok = (stage_ok & ~(1u << stg)) | (ok << stg);
-    if (!ok) fill_bad(stg);  // warp-uniform (ok comes from a ballot)
     if (lane == src) {
       uint64_t* bar = &bars[stg];
       fence_proxy_async_smem();  // the warp's reads of this stage precede the copy
@@ -948,70 +945,33 @@ __global__ void __launch_bounds__(Shape<FMT, D>::NW * 32, 1)
         F::issue(ring + stg * F::STAGE, bar, &mk, &mv, &mks, &mvs, cur_h, cur_blk);
       } else {
         set_err(p.d_err, kErrBlockId);
-        mbar_arrive(bar);  // completes the phase with no data
+        mbar_arrive(bar);  // completes the phase with no data; the page is skipped
       }
     }
   };
   // Prologue: lane i fills stage i with local item i (its own cur_blk), the
   // lanes' copies issued together rather than one after another.
-  int issued = min(NSW, n_local);  // local items whose copies have been issued
   {
-    stage_ok = ok_win & ((1u << issued) - 1u);
-    for (int i = 0; i < issued; ++i)  // rare: zero-fill the stages of bad ids
-      if (!((ok_win >> i) & 1u)) fill_bad(i);
-    if (lane < issued) {
+    const int n0 = min(NSW, n_local);
+    stage_ok = ok_win & ((1u << n0) - 1u);
+    if (lane < n0) {
       uint64_t* bar = &bars[lane];
       if ((ok_win >> lane) & 1u) {
         F::issue(ring + lane * F::STAGE, bar, &mk, &mv, &mks, &mvs, cur_h, cur_blk);
       } else {
         set_err(p.d_err, kErrBlockId);
-        mbar_arrive(bar);  // completes the phase with no data
+        mbar_arrive(bar);  // completes the phase with no data; the page is skipped
       }
     }
   }
 
-  // Ring of the warp's local items: item i sits in stage i % NSW and its copy
-  // completes barrier phase (i / NSW) & 1.  A stage is held from the wait for
-  // its item until that item's V has been read, one loop trip later, and is
-  // then refilled with the next item not yet issued.
-  int k_base = 0, j = 0;  // j = this warp's next local item to wait for
+  int k_base = 0, j = 0;  // j = this warp's next local item
   int st = 0, ph = 0;     // its stage (j % NSW) and barrier phase parity ((j / NSW) & 1)
-  bool dead = false;      // a bounded wait expired: this warp reads no more pages
-  // Waits for item j (all lanes agree, so the warp stays converged).  If the
-  // wait expires: report it, wait (bounded) for the copies still in flight
-  // (items j+1 .. issued-1) and stop reading pages.
-  auto wait_item = [&]() -> bool {
-    if (__all_sync(0xffffffffu, mbar_wait_bounded(&bars[st], ph))) return true;
-    if (lane == 0) set_err(p.d_err, kErrTimeout);
-    for (int i = j + 1; i < issued; ++i) mbar_wait_bounded(&bars[i % NSW], (i / NSW) & 1);
-    dead = true;
-    return false;
-  };
-  auto advance = [&]() {
-    ++j;
-    if (++st == NSW) {
-      st = 0;
-      ph ^= 1;
-    }
-  };
-  // Refill the stage of a consumed item with the next item not yet issued.
-  auto refill = [&](int stg) {
-    __syncwarp();  // every lane's reads of the stage are done
-    if (issued < n_local) {
-      issue(issued, stg);
-      ++issued;
-    }
-  };
-  // S^T = K Q^T of the page in stage stg on tensor cores (two accumulator
-  // chains): the raw scores r[i] = q . k_code of this thread's (token, head)
-  // pairs (tokens gid, gid+8; heads 2tig, 2tig+1).
   // FP8 attention: S[head][token] = Q_hat K^T on E4M3 tensor cores, the K
-  // codes read straight from the stage as the B operand (column = token gid
+  // codes as read from the stage forming the B operand (column = token gid
   // for tokens 0-7, gid+8 for tokens 8-15); this thread gets head gid's
   // scores of tokens 2tig, 2tig+1 (r[0], r[1]) and 2tig+8, 2tig+9 (r[2], r[3]).
-  auto qk_page = [&](int stg, float r[4]) {
-    typename F::Raw raw;
-    F::load_raw_k(ring + stg * F::STAGE, gid, tig, raw);
+  auto qk_page = [&](const typename F::Raw& raw, float r[4]) {
     if constexpr (QP) {
       constexpr int NR = sizeof(raw.k) / sizeof(raw.k[0]) / 2;  // uint4 per row
       float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
@@ -1091,22 +1051,31 @@ __global__ void __launch_bounds__(Shape<FMT, D>::NW * 32, 1)
     // masked (only the unit's relative page 0 can hold such tokens)
     const int n_skip = (p.window > 0 && len > p.window) ? len - p.window - first * kPage : 0;
 
-    // Softmax of page k, part 1: mask the raw scores r of the tokens outside
-    // [t_lo, t_hi) of the page and turn them into exponents e = s - m + kPLog2
-    // (s = c_log2 r).  The running max m moves only when a score passes m +
+    // Softmax of a page, part 1: turn the raw scores r into exponents e = s -
+    // m + kPLog2 (s = c_log2 r).  The running max m moves only when a score passes m +
     // kRescaleGap (one vote, no reduction, on most pages); p = 2^(s - m) then
     // stays <= 2^kRescaleGap, which keeps P = p 2^kPLog2 inside f16.
-    auto softmax_e = [&](float r[4], int t_lo, int t_hi, float e[4]) {
-      if constexpr (QP) {
-        // FP8 attention: r holds head gid's raw scores of tokens 2tig,
-        // 2tig+1, 2tig+8, 2tig+9.  P is quantized against the page's own
-        // largest score mp, p = 2^(s - mp), P_hat = E4M3(p / prob_scale);
-        // the page then enters the running sums with weight f = 2^(mp - mq).
+    // Raw scores of the tokens outside [t_lo, t_hi) of the page become -inf
+    // (only edge pages: the window's first page, the segment's last page, a
+    // page with a bad block id).
+    auto mask_scores = [&](float r[4], int t_lo, int t_hi) {
+      if constexpr (QP) {  // r: tokens 2tig, 2tig+1, 2tig+8, 2tig+9
         const int t0 = 2 * tig;
         if (!(t0 >= t_lo && t0 < t_hi)) r[0] = -kInf;
         if (!(t0 + 1 >= t_lo && t0 + 1 < t_hi)) r[1] = -kInf;
         if (!(t0 + 8 >= t_lo && t0 + 8 < t_hi)) r[2] = -kInf;
         if (!(t0 + 9 >= t_lo && t0 + 9 < t_hi)) r[3] = -kInf;
+      } else {  // r: tokens gid (r[0], r[1]) and gid+8 (r[2], r[3])
+        if (!(gid >= t_lo && gid < t_hi)) r[0] = r[1] = -kInf;
+        if (!(gid + 8 >= t_lo && gid + 8 < t_hi)) r[2] = r[3] = -kInf;
+      }
+    };
+    auto softmax_e = [&](float r[4], float e[4]) {
+      if constexpr (QP) {
+        // FP8 attention: r holds head gid's raw scores of tokens 2tig,
+        // 2tig+1, 2tig+8, 2tig+9.  P is quantized against the page's own
+        // largest score mp, p = 2^(s - mp), P_hat = E4M3(p / prob_scale);
+        // the page then enters the running sums with weight f = 2^(mp - mq).
         float rmax = fmaxf(fmaxf(r[0], r[1]), fmaxf(r[2], r[3]));
         rmax = fmaxf(rmax, __shfl_xor_sync(0xffffffffu, rmax, 1));
         rmax = fmaxf(rmax, __shfl_xor_sync(0xffffffffu, rmax, 2));
@@ -1143,8 +1112,6 @@ __global__ void __launch_bounds__(Shape<FMT, D>::NW * 32, 1)
         e[2] = __shfl_sync(0xffffffffu, f, 8 * tig + 4);  // weight of head 2tig+1
         return;
       }
-      if (!(gid >= t_lo && gid < t_hi)) r[0] = r[1] = -kInf;
-      if (!(gid + 8 >= t_lo && gid + 8 < t_hi)) r[2] = r[3] = -kInf;
       e[0] = fmaf(r[0], c_log2, n0);
       e[1] = fmaf(r[1], c_log2, n1);
       e[2] = fmaf(r[2], c_log2, n0);
@@ -1179,47 +1146,56 @@ __global__ void __launch_bounds__(Shape<FMT, D>::NW * 32, 1)
         e[3] = s3 + n1;
       }
     };
-    // Softmax of a page, part 2, and O^T += V^T P^T with the page's V read from
-    // stage stg.  Tokens at or past n_valid are zeroed in V (only the unit's
-    // last page can hold unwritten slots, possibly NaN codes).
-    auto pv_page = [&](const float e[4], int stg, int n_valid) {
+    // The V operand of a page's PV product, from the stage words in registers.
+    // FP8 attention: per head-dim row, the codes of tokens 2tig, 2tig+1,
+    // 2tig+8, 2tig+9 (the token order of P_hat), a byte transpose of the
+    // thread's four token rows: va[jj][0], va[jj][1] (rows gid, gid+8).
+    auto prep_v = [&](const typename F::Raw& raw, uint32_t va[MT][4]) {
       if constexpr (QP) {
-        // FP8 attention: O^T += f * (V^T P_hat^T) on E4M3 tensor cores.  The A
-        // operand holds, per head-dim row, the codes of tokens 2tig, 2tig+1,
-        // 2tig+8, 2tig+9 (the token order of P_hat): a byte transpose of the
-        // thread's four token rows.
-        typename F::Raw raw;
-        F::load_raw_v(ring + stg * F::STAGE, gid, tig, raw);
         constexpr int NWD = D / 32;  // 32-bit words of a thread's run of one token row
-        uint32_t x[4][NWD];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const uint32_t* w = reinterpret_cast<const uint32_t*>(&raw.v[i]);
-#pragma unroll
-          for (int k = 0; k < NWD; ++k) x[i][k] = w[k];
-        }
-        uint32_t msk = 0xFFFFFFFFu;
-        if (n_valid < kPage)  // unwritten slots may hold NaN codes
-          msk = (2 * tig < n_valid ? 0x000000FFu : 0u) | (2 * tig + 1 < n_valid ? 0x0000FF00u : 0u) |
-                (2 * tig + 8 < n_valid ? 0x00FF0000u : 0u) |
-                (2 * tig + 9 < n_valid ? 0xFF000000u : 0u);
-        const uint32_t pq = __float_as_uint(e[0]);
 #pragma unroll
         for (int k = 0; k < NWD; ++k) {
-          const uint32_t xyl = prmt(x[0][k], x[1][k], 0x5140), ztl = prmt(x[2][k], x[3][k], 0x5140);
-          const uint32_t xyh = prmt(x[0][k], x[1][k], 0x7362), zth = prmt(x[2][k], x[3][k], 0x7362);
-          const uint32_t a[4] = {prmt(xyl, ztl, 0x5410) & msk, prmt(xyl, ztl, 0x7632) & msk,
-                                 prmt(xyh, zth, 0x5410) & msk, prmt(xyh, zth, 0x7632) & msk};
+          uint32_t x[4];
 #pragma unroll
-          for (int hh = 0; hh < 2; ++hh) {  // m-tile 2k + hh: head-dim bytes 2hh, 2hh+1 of word k
-            const int jj = 2 * k + hh;
-            float acc[4];
-            mma_e4m3_k16(acc, a[2 * hh], a[2 * hh + 1], pq);
-            o[jj][0] = fmaf(e[1], acc[0], o[jj][0]);
-            o[jj][1] = fmaf(e[2], acc[1], o[jj][1]);
-            o[jj][2] = fmaf(e[1], acc[2], o[jj][2]);
-            o[jj][3] = fmaf(e[2], acc[3], o[jj][3]);
+          for (int i = 0; i < 4; ++i) x[i] = reinterpret_cast<const uint32_t*>(&raw.v[i])[k];
+          const uint32_t xyl = prmt(x[0], x[1], 0x5140), ztl = prmt(x[2], x[3], 0x5140);
+          const uint32_t xyh = prmt(x[0], x[1], 0x7362), zth = prmt(x[2], x[3], 0x7362);
+          va[2 * k][0] = prmt(xyl, ztl, 0x5410);  // head-dim byte 0 of word k
+          va[2 * k][1] = prmt(xyl, ztl, 0x7632);  // byte 1
+          va[2 * k + 1][0] = prmt(xyh, zth, 0x5410);  // byte 2
+          va[2 * k + 1][1] = prmt(xyh, zth, 0x7632);  // byte 3
+        }
+      } else {
+        F::conv_v(raw, va);
+      }
+    };
+    // Softmax of a page, part 2, and O^T += V^T P^T.  Tokens at or past
+    // n_valid are zeroed in V (only the unit's last page can hold unwritten
+    // slots, possibly NaN codes).
+    auto pv_page = [&](const float e[4], uint32_t va[MT][4], int n_valid) {
+      if constexpr (QP) {
+        // FP8 attention: O^T += f * (V^T P_hat^T) on E4M3 tensor cores, each
+        // page into a fresh accumulator weighted by its f.
+        if (n_valid < kPage) {
+          const uint32_t msk =
+              (2 * tig < n_valid ? 0x000000FFu : 0u) | (2 * tig + 1 < n_valid ? 0x0000FF00u : 0u) |
+              (2 * tig + 8 < n_valid ? 0x00FF0000u : 0u) |
+              (2 * tig + 9 < n_valid ? 0xFF000000u : 0u);
+#pragma unroll
+          for (int jj = 0; jj < MT; ++jj) {
+            va[jj][0] &= msk;
+            va[jj][1] &= msk;
           }
+        }
+        const uint32_t pq = __float_as_uint(e[0]);
+#pragma unroll
+        for (int jj = 0; jj < MT; ++jj) {
+          float acc[4];
+          mma_e4m3_k16(acc, va[jj][0], va[jj][1], pq);
+          o[jj][0] = fmaf(e[1], acc[0], o[jj][0]);
+          o[jj][1] = fmaf(e[2], acc[1], o[jj][1]);
+          o[jj][2] = fmaf(e[1], acc[2], o[jj][2]);
+          o[jj][3] = fmaf(e[2], acc[3], o[jj][3]);
         }
         return;
       }
@@ -1227,10 +1203,6 @@ __global__ void __launch_bounds__(Shape<FMT, D>::NW * 32, 1)
                   q3 = fast_exp2(e[3]);
       l0 += q0 + q2;  // l and O carry the factor 2^kPLog2, removed at normalisation
       l1 += q1 + q3;
-      typename F::Raw raw;
-      uint32_t va[MT][4];
-      F::load_raw_v(ring + stg * F::STAGE, gid, tig, raw);
-      F::conv_v(raw, va);
       if (n_valid < kPage) {
         const uint32_t m01 = (2 * tig < n_valid ? 0x0000FFFFu : 0u) |
                              (2 * tig + 1 < n_valid ? 0xFFFF0000u : 0u);
@@ -1270,47 +1242,186 @@ __global__ void __launch_bounds__(Shape<FMT, D>::NW * 32, 1)
         mma16816<F::kBF16>(o[jj], va[jj], bl0, bl1);
       }
     };
-    // Valid token range [t_lo, t_hi) of page k (before the last-page cut).
-    auto t_lo_of = [&](int k, bool valid) {
-      return !valid ? kPage : (n_skip > 0 && ps == 0 && k == k_base) ? n_skip : 0;
-    };
 
-    // Software pipeline over this warp's pages of the segment: while page C's
-    // softmax and PV run, page N's K is read and its QK issued, two
-    // independent dependency chains in one straight-line block.
-    int kc = warp + j * NW;  // this warp's first page of the segment
-    if (!dead && kc < k_end && wait_item()) {
-      float rc[4];
-      bool vc = (stage_ok >> st) & 1u;
-      int stc = st;
-      qk_page(stc, rc);
-      advance();
-      for (int kn = kc + NW; kn < k_end; kn += NW) {
-        float ec[4];
-        softmax_e(rc, t_lo_of(kc, vc), kPage, ec);  // C is not the segment's last page
-        if (!wait_item()) break;
-        const bool vn = (stage_ok >> st) & 1u;
-        const int stn = st;
-        float rn[4];
-        qk_page(stn, rn);        // chain 1: page N
-        pv_page(ec, stc, kPage);  // chain 2: page C
-        refill(stc);
-        advance();
-        kc = kn;
-        stc = stn;
-        vc = vn;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) rc[i] = rn[i];
+    if constexpr (QP) {
+      // FP8 attention: the same page loop, the page's work in the lambdas above
+      for (int k = warp + j * NW; k < k_end; k += NW, ++j) {
+        if (!__all_sync(0xffffffffu, mbar_wait_bounded(&bars[st], ph))) {
+          if (lane == 0) set_err(p.d_err, kErrTimeout);
+          for (int i = j + 1; i < j + NSW && i < n_local; ++i)  // drain copies in flight
+            mbar_wait_bounded(&bars[i % NSW], (i / NSW) & 1);
+          j = n_local;
+          break;
+        }
+        const bool valid = (stage_ok >> st) & 1u;
+        typename F::Raw raw;
+        if (valid) {
+          F::load_raw_k(ring + st * F::STAGE, gid, tig, raw);
+          F::load_raw_v(ring + st * F::STAGE, gid, tig, raw);
+        }
+        __syncwarp();
+        if (j + NSW < n_local) issue(j + NSW, st);  // item j + NSW reuses stage st
+        if (++st == NSW) {
+          st = 0;
+          ph ^= 1;
+        }
+        if (!valid) continue;
+        float r[4], e[4];
+        uint32_t va[MT][4];
+        qk_page(raw, r);
+        prep_v(raw, va);
+        // valid tokens [t_lo, t_hi) of an edge page: the window's first page
+        // starts late, the segment's last page may end early
+        const bool first_w = n_skip > 0 && ps == 0 && k == k_base;
+        int t_hi = kPage;
+        if (first_w || k == k_end - 1) {
+          t_hi = (k == k_end - 1 && n_last < kPage) ? n_last : kPage;
+          mask_scores(r, first_w ? n_skip : 0, t_hi);
+        }
+        softmax_e(r, e);
+        pv_page(e, va, t_hi);
       }
-      if (!dead) {  // the warp's last page of the segment
-        const int t_hi = (kc == k_end - 1 && n_last < kPage) ? n_last : kPage;
-        float ec[4];
-        softmax_e(rc, t_lo_of(kc, vc), t_hi, ec);
-        pv_page(ec, stc, t_hi);
-        refill(stc);
+    } else {
+      for (int k = warp + j * NW; k < k_end; k += NW, ++j) {
+        const uint8_t* sp = ring + st * F::STAGE;
+        // all lanes agree on the outcome so the warp stays converged
+        if (!__all_sync(0xffffffffu, mbar_wait_bounded(&bars[st], ph))) {
+          if (lane == 0) set_err(p.d_err, kErrTimeout);
+          for (int i = j + 1; i < j + NSW && i < n_local; ++i)  // drain copies in flight
+            mbar_wait_bounded(&bars[i % NSW], (i / NSW) & 1);
+          j = n_local;
+          break;
+        }
+        const bool valid = (stage_ok >> st) & 1u;
+
+        // The stage's words go to registers first, so the stage is refilled with
+        // local item j + NSW before any decode or math on this one (for BF16
+        // head_dim 128, after the QK product: see kLateV).
+        typename F::Raw raw;
+        uint32_t ka[KS][4], va[MT][4];
+        float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
+        // ---- S^T = K Q^T on tensor cores (two accumulator chains)
+        auto qk = [&]() {
+          F::conv_k(raw, ka);
+  #pragma unroll
+          for (int s = 0; s < KS; ++s) {
+            if (s & 1)
+              mma16816<F::kBF16>(sb, ka[s], qb[s][0], qb[s][1]);
+            else
+              mma16816<F::kBF16>(sa, ka[s], qb[s][0], qb[s][1]);
+          }
+        };
+        if constexpr (F::kLateV) {
+          if (valid) {
+            F::load_raw_k(sp, gid, tig, raw);
+            qk();
+            F::load_raw_v(sp, gid, tig, raw);
+          }
+        } else if (valid) {
+          F::load_raw_k(sp, gid, tig, raw);
+          F::load_raw_v(sp, gid, tig, raw);
+        }
+        __syncwarp();
+        if (j + NSW < n_local) issue(j + NSW, st);  // item j + NSW reuses stage st
+        if (++st == NSW) {
+          st = 0;
+          ph ^= 1;
+        }
+        if (!valid) continue;
+        if constexpr (!F::kLateV) qk();
+        F::conv_v(raw, va);
+
+        // raw scores r = q . k_code (the scale c_log2 is applied below)
+        float r0 = sa[0] + sb[0], r1 = sa[1] + sb[1], r2 = sa[2] + sb[2], r3 = sa[3] + sb[3];
+        if (k == k_end - 1 && n_last < kPage) {  // last, partial page: mask tokens past the length
+          const int n_valid = n_last;
+          if (gid >= n_valid) r0 = r1 = -kInf;
+          if (gid + 8 >= n_valid) r2 = r3 = -kInf;
+          const uint32_t m01 = (2 * tig < n_valid ? 0x0000FFFFu : 0u) |
+                               (2 * tig + 1 < n_valid ? 0xFFFF0000u : 0u);
+          const uint32_t m23 = (2 * tig + 8 < n_valid ? 0x0000FFFFu : 0u) |
+                               (2 * tig + 9 < n_valid ? 0xFFFF0000u : 0u);
+  #pragma unroll
+          for (int jj = 0; jj < MT; ++jj) {  // unwritten slots may hold NaN codes
+            va[jj][0] &= m01;
+            va[jj][1] &= m01;
+            va[jj][2] &= m23;
+            va[jj][3] &= m23;
+          }
+        }
+        if (n_skip > 0 && ps == 0 && k == k_base) {  // window's first page: tokens before it
+          if (gid < n_skip) r0 = r1 = -kInf;
+          if (gid + 8 < n_skip) r2 = r3 = -kInf;
+        }
+
+        // ---- online softmax (log2 domain); this thread: heads 2tig, 2tig+1.
+        // The running max m moves only when a score passes m + kRescaleGap
+        // (one vote, no reduction, on most pages); p = 2^(s - m) then stays
+        // <= 2^kRescaleGap, which keeps P = p * 2^kPLog2 inside f16.
+        // e = s - m + kPLog2 with s = c_log2 * r: 2^e = p * 2^kPLog2 = P as fed to the MMA
+        float e0 = fmaf(r0, c_log2, n0), e1 = fmaf(r1, c_log2, n1);
+        float e2 = fmaf(r2, c_log2, n0), e3 = fmaf(r3, c_log2, n1);
+        if (__any_sync(0xffffffffu, e0 > kETop || e2 > kETop || e1 > kETop || e3 > kETop)) {
+          const float s0 = r0 * c_log2, s1 = r1 * c_log2, s2 = r2 * c_log2, s3 = r3 * c_log2;
+          float mx0 = fmaxf(s0, s2), mx1 = fmaxf(s1, s3);
+  #pragma unroll
+          for (int off = 4; off < 32; off <<= 1) {
+            mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+            mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+          }
+          const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
+          const float a0 = fast_exp2(m0 - mn0), a1 = fast_exp2(m1 - mn1);  // 0 while m = -inf
+          l0 *= a0;
+          l1 *= a1;
+  #pragma unroll
+          for (int jj = 0; jj < MT; ++jj) {
+            o[jj][0] *= a0;
+            o[jj][1] *= a1;
+            o[jj][2] *= a0;
+            o[jj][3] *= a1;
+          }
+          m0 = mn0;
+          m1 = mn1;
+          n0 = kPLog2 - m0;
+          n1 = kPLog2 - m1;
+          e0 = s0 + n0;
+          e1 = s1 + n1;
+          e2 = s2 + n0;
+          e3 = s3 + n1;
+        }
+        const float q0 = fast_exp2(e0), q1 = fast_exp2(e1), q2 = fast_exp2(e2), q3 = fast_exp2(e3);
+        l0 += q0 + q2;  // l and O carry the factor 2^kPLog2, removed at normalisation
+        l1 += q1 + q3;
+
+        // ---- P^T fragments: high part + residual, transposed in registers
+        uint32_t x0h, x1h, x0l, x1l;
+        float h0, h1, h2, h3;  // the high parts as fp32
+        if constexpr (F::kBF16) {
+          x0h = pack_bf16x2(q0, q1);
+          x1h = pack_bf16x2(q2, q3);
+          unpack_bf16x2(x0h, h0, h1);
+          unpack_bf16x2(x1h, h2, h3);
+          x0l = pack_bf16x2(q0 - h0, q1 - h1);
+          x1l = pack_bf16x2(q2 - h2, q3 - h3);
+        } else {
+          x0h = pack_f16x2(q0, q1);
+          x1h = pack_f16x2(q2, q3);
+          unpack_f16x2(x0h, h0, h1);
+          unpack_f16x2(x1h, h2, h3);
+          x0l = pack_f16x2(q0 - h0, q1 - h1);
+          x1l = pack_f16x2(q2 - h2, q3 - h3);
+        }
+        const uint32_t bh0 = movmatrix_t(x0h), bh1 = movmatrix_t(x1h);
+        const uint32_t bl0 = movmatrix_t(x0l), bl1 = movmatrix_t(x1l);
+
+        // ---- O^T += V^T P^T
+  #pragma unroll
+        for (int jj = 0; jj < MT; ++jj) {
+          mma16816<F::kBF16>(o[jj], va[jj], bh0, bh1);
+          mma16816<F::kBF16>(o[jj], va[jj], bl0, bl1);
+        }
       }
     }
-    if (dead) j = n_local;  // no further segment reads a page
     k_base = k_end;
 
     // ---- segment end: warp partials -> shared slots, merged by the CTA
