@@ -584,12 +584,14 @@ def main():
         extras["fp8_attention"] = fq
 
         # BF16 vs FP8 vs NVFP4 decode on the byte-heavy 4 x 126,976-token
-        # D=128 cache and on the 1 x 65,536-token D=64 workload
+        # D=128 cache (and the 3-bit PQ3 codec, which needs D=128) and on the
+        # 1 x 65,536-token D=64 workload
         for key, name, reps in (("formats_4x127k", "agents-fp8-4x127k", Kx),
                                 ("formats_1x64k", "nvfp4-1x64k", K)):
             wf = wl.WORKLOADS[name]
             fm = {}
-            for fmt in ("bf16", "fp8", "nvfp4"):
+            fmts = ("bf16", "fp8", "nvfp4", "pq3") if wf.D == 128 else ("bf16", "fp8", "nvfp4")
+            for fmt in fmts:
                 s2 = DecodeScenario(wf, fmt=fmt, device="cuda")
                 (dms,), _ = timer.run([s2.decode], reps, W)
                 assert int(s2.err.item()) == 0

@@ -66,6 +66,28 @@
  *          to +-6; all codes +0 when that divisor is 0);
  *          value = E2M1_value(code) * E4M3_value(sb) * g.
  *   BF16 : scales are ignored and may be NULL.
+ *
+ * KVQ_FMT_PQ3 ("AMD MI300X - KV Cache Compression Benchmark", "Key Results":
+ * 3-bit methods with one 52-byte block per 128-element vector, 4.923x against
+ * FP16; PlanarQuant's rotation needs 256 FMAs; the repository generates a
+ * Lloyd-Max codebook).  Each 128-element head vector x (one token, one KV
+ * head, K or V) is stored as its fp32 L2 norm and 128 3-bit indices:
+ *   u = x / |x|; y = R u with R = 64 planar rotations of the coordinate
+ *   pairs (2j, 2j+1) by (cos_j, sin_j); index_i = the nearest of 8 codebook
+ *   values c_0 < ... < c_7 to y_i; value = |x| * R^T c[index].
+ * The encode's fp32 steps are fixed, so indices are exact: sum of squares as
+ * a pairwise tree in index order, sqrt and division rounded to nearest,
+ * y_2j = fma(cos_j, u_2j, -(sin_j * u_2j+1)), y_2j+1 = fma(sin_j, u_2j,
+ * cos_j * u_2j+1), index = the number of thresholds (c_k + c_k+1) / 2 below
+ * y; an all-zero x stores norm 0 and indices 0.
+ *   Head page (832 bytes): 16 fp32 norms, then 16 rows of 48 bytes; index i
+ *   of a row sits in bits [3i, 3i+3) of the row's little-endian bit string.
+ *   The "scale" of a PQ3 tensor (d_k_scale, d_v_scale) is a device array of
+ *   136 fp32: the 8 codebook values (f16-representable, ascending; see
+ *   kv_pq3_codebook), then the 64 (cos, sin) pairs.
+ *   kv_decode_attention, its window mode, kv_quantize_write, kv_dequantize
+ *   and kv_cache_bytes accept PQ3; kv_prefill_attention and
+ *   kv_scale_from_absmax(_device) do not (KVQ_ERR_UNSUPPORTED).
  */
 #ifndef KVQ_H
 #define KVQ_H
@@ -82,7 +104,8 @@ extern "C" {
 typedef enum kvq_format {
   KVQ_FMT_BF16 = 0,
   KVQ_FMT_FP8_E4M3 = 1,
-  KVQ_FMT_NVFP4 = 2
+  KVQ_FMT_NVFP4 = 2,
+  KVQ_FMT_PQ3 = 3 /* 3-bit planar-rotation codec, head_dim 128 only (see below) */
 } kvq_format;
 
 typedef enum kvq_status {
@@ -123,7 +146,8 @@ const char* kvq_last_error(void);
 
 /* Bytes of ONE of the two cache buffers (K or V) for the given geometry:
  * num_blocks * num_kv_heads * head-page bytes, a head page being 32*head_dim
- * bytes (BF16), 16*head_dim (FP8) or 9*head_dim (NVFP4). */
+ * bytes (BF16), 16*head_dim (FP8), 9*head_dim (NVFP4) or 832 (PQ3, head_dim
+ * 128). */
 kvq_status kv_cache_bytes(int32_t fmt, int64_t num_blocks, int32_t num_kv_heads,
                           int32_t head_dim, int64_t* bytes);
 
@@ -134,6 +158,14 @@ kvq_status kv_cache_bytes(int32_t fmt, int64_t num_blocks, int32_t num_kv_heads,
  *   BF16 : 1.
  * amax must be finite and >= 0. */
 kvq_status kv_scale_from_absmax(int32_t fmt, float amax, float* scale);
+
+/* Host, pure.  The PQ3 codebook: the 8-level Lloyd-Max quantizer of N(0, 1/128)
+ * (one coordinate of a random unit vector in 128 dimensions, Gaussian
+ * approximation; "AMD MI300X - KV Cache Compression Benchmark", repository
+ * structure: Lloyd-Max solver and codebook generator), each value rounded to
+ * the nearest f16, written to cb[8] in ascending order.  KVQ_ERR_INVALID_ARG
+ * if cb is NULL. */
+kvq_status kv_pq3_codebook(float* cb);
 
 /* Device version of kv_scale_from_absmax: reads *d_amax, writes *d_scale
  * (bit-identical to the host function), so calibration, scale and

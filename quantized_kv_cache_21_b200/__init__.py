@@ -7,9 +7,11 @@ current CUDA stream).  Every step of the computation runs in the library's
 CUDA kernels; there is no Python or CPU fallback, and importing the compute
 functions without the built library raises.
 
-Formats: ``"bf16"``, ``"fp8"`` (OCP E4M3 with a per-layer fp32 scale) and
+Formats: ``"bf16"``, ``"fp8"`` (OCP E4M3 with a per-layer fp32 scale),
 ``"nvfp4"`` (16-element E2M1 blocks along head_dim, E4M3 block scales and an
-fp32 per-tensor scale; 4.5 bits per element).
+fp32 per-tensor scale; 4.5 bits per element) and ``"pq3"`` (3-bit
+planar-rotation codec of 128-element vectors, 52 bytes each; its "scale" is a
+136-float parameter block, see ``pq3_params``).
 """
 from __future__ import annotations
 
@@ -20,7 +22,7 @@ import torch
 
 from .build import LIB as _LIB_PATH
 
-FORMATS = {"bf16": 0, "fp8": 1, "nvfp4": 2}
+FORMATS = {"bf16": 0, "fp8": 1, "nvfp4": 2, "pq3": 3}
 BLOCK_SIZE = 16
 
 DERR_BLOCK_ID = 0x1
@@ -30,6 +32,7 @@ DERR_SEQ_LEN = 0x8
 DERR_TIMEOUT = 0x10
 
 EXPORTS = ("kvq_status_string", "kvq_last_error", "kv_cache_bytes", "kv_scale_from_absmax",
+           "kv_pq3_codebook",
            "kv_scale_from_absmax_device", "kv_calibrate_absmax", "kv_quantize_write",
            "kv_decode_workspace_size", "kv_decode_attention", "kv_decode_attention_static_ws",
            "kv_decode_attention_window", "kv_decode_workspace_size_window",
@@ -67,6 +70,7 @@ def lib() -> ctypes.CDLL:
         sigs = {
             "kv_cache_bytes": [i32, i64, i32, i32, ctypes.POINTER(i64)],
             "kv_scale_from_absmax": [i32, f32, ctypes.POINTER(f32)],
+            "kv_pq3_codebook": [P],
             "kv_scale_from_absmax_device": [i32, P, P, P],
             "kv_calibrate_absmax": [P, i64, P, P],
             "kv_quantize_write": [i32, P, P, i64, P, P, i32, i32, CP, P, P, P, P],
@@ -154,6 +158,22 @@ def kv_scale_from_absmax(fmt, amax: float) -> float:
     out = ctypes.c_float()
     _check(lib().kv_scale_from_absmax(_fmt(fmt), float(amax), ctypes.byref(out)))
     return out.value
+
+
+def kv_pq3_codebook() -> list:
+    """The PQ3 codebook (8 ascending f16-representable values, see include/kvq.h)."""
+    out = (ctypes.c_float * 8)()
+    _check(lib().kv_pq3_codebook(ctypes.cast(out, ctypes.c_void_p)))
+    return list(out)
+
+
+def pq3_params(cos_sin, device="cuda") -> torch.Tensor:
+    """The 136-float PQ3 parameter block of one tensor on the device: the
+    codebook, then the 64 (cos, sin) pairs of its planar rotation."""
+    rot = torch.as_tensor(cos_sin, dtype=torch.float32).reshape(-1)
+    assert rot.numel() == 128
+    cb = torch.tensor(kv_pq3_codebook(), dtype=torch.float32)
+    return torch.cat([cb, rot]).to(device)
 
 
 def kv_scale_from_absmax_device(fmt, d_amax: torch.Tensor, d_scale: torch.Tensor, stream=None):

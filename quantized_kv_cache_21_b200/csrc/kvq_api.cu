@@ -2,8 +2,11 @@
 // context-split plan, TMA descriptors for the paged cache, and launches.
 #include <cudaTypedefs.h>
 #include <math.h>
+
+#include <cmath>
 #include <stdarg.h>
 #include <stdio.h>
+#include <string.h>
 
 #include <atomic>
 #include <mutex>
@@ -53,17 +56,20 @@ bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p
 int64_t head_page_bytes(int fmt, int D) {
   if (fmt == KVQ_FMT_BF16) return 32LL * D;
   if (fmt == KVQ_FMT_FP8_E4M3) return 16LL * D;
+  if (fmt == KVQ_FMT_PQ3) return 16LL * 52;  // per token: fp32 norm + 48 index bytes
   return 9LL * D;
 }
 
 kvq_status check_cache(int32_t fmt, const kvq_cache* c) {
-  if (fmt < 0 || fmt > 2) return fail(KVQ_ERR_UNSUPPORTED, "unknown format %d", fmt);
+  if (fmt < 0 || fmt > 3) return fail(KVQ_ERR_UNSUPPORTED, "unknown format %d", fmt);
   if (!c) return fail(KVQ_ERR_INVALID_ARG, "cache is NULL");
   if (c->fmt != fmt) return fail(KVQ_ERR_INVALID_ARG, "cache format %d != fmt %d", c->fmt, fmt);
   if (c->block_size != KVQ_BLOCK_SIZE)
     return fail(KVQ_ERR_UNSUPPORTED, "block_size %d (only 16)", c->block_size);
   if (c->head_dim != 64 && c->head_dim != 128)
     return fail(KVQ_ERR_UNSUPPORTED, "head_dim %d (64 or 128)", c->head_dim);
+  if (fmt == KVQ_FMT_PQ3 && c->head_dim != 128)
+    return fail(KVQ_ERR_UNSUPPORTED, "PQ3 needs head_dim 128 (got %d)", c->head_dim);
   if (c->num_kv_heads < 1) return fail(KVQ_ERR_INVALID_ARG, "num_kv_heads %d", c->num_kv_heads);
   if (c->num_blocks < 1 || c->num_blocks > 0x7fffffffLL)
     return fail(KVQ_ERR_INVALID_ARG, "num_blocks %lld", (long long)c->num_blocks);
@@ -87,7 +93,7 @@ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 kvq_status make_plan(int32_t fmt, int32_t B, int32_t Hq, int32_t Hkv, int32_t D,
                      int32_t max_seq_len, int32_t num_splits, Plan* pl, int32_t window = 0) {
   kvq::DecodeConfig cfg;
-  if (fmt < 0 || fmt > 2 || !kvq::decode_config(fmt, D, &cfg))
+  if (fmt < 0 || fmt > 3 || !kvq::decode_config(fmt, D, &cfg))
     return fail(KVQ_ERR_UNSUPPORTED, "format %d / head_dim %d", fmt, D);
   if (B < 0 || Hkv < 1 || Hq < Hkv || Hq % Hkv != 0)
     return fail(KVQ_ERR_INVALID_ARG, "num_seqs %d, num_q_heads %d, num_kv_heads %d", B, Hq, Hkv);
@@ -174,6 +180,11 @@ kvq_status encode(CUtensorMap* m, CUtensorMapDataType dt, cuuint32_t rank, void*
 // [1] = NVFP4 block-scale run of a head page (same as [0] otherwise).
 kvq_status make_maps(int fmt, const kvq_cache* c, void* buf, CUtensorMap* tile, CUtensorMap* sf) {
   const cuuint64_t D = c->head_dim, H = c->num_kv_heads, nb = c->num_blocks;
+  if (fmt == KVQ_FMT_PQ3) {  // head pages are fetched whole with bulk copies: no map
+    memset(tile, 0, sizeof(*tile));
+    memset(sf, 0, sizeof(*sf));
+    return KVQ_OK;
+  }
   if (fmt == KVQ_FMT_FP8_E4M3) {
     const cuuint64_t dims[4] = {D, 16, H, nb};
     const cuuint64_t str[3] = {D, 16 * D, 16 * D * H};
@@ -292,15 +303,54 @@ const char* kvq_last_error(void) { return g_err; }
 
 kvq_status kv_cache_bytes(int32_t fmt, int64_t num_blocks, int32_t num_kv_heads,
                           int32_t head_dim, int64_t* bytes) {
-  if (fmt < 0 || fmt > 2) return fail(KVQ_ERR_UNSUPPORTED, "unknown format %d", fmt);
+  if (fmt < 0 || fmt > 3) return fail(KVQ_ERR_UNSUPPORTED, "unknown format %d", fmt);
   if (head_dim != 64 && head_dim != 128) return fail(KVQ_ERR_UNSUPPORTED, "head_dim %d", head_dim);
+  if (fmt == KVQ_FMT_PQ3 && head_dim != 128)
+    return fail(KVQ_ERR_UNSUPPORTED, "PQ3 needs head_dim 128 (got %d)", head_dim);
   if (num_blocks < 0 || num_kv_heads < 1 || !bytes)
     return fail(KVQ_ERR_INVALID_ARG, "num_blocks/num_kv_heads/bytes");
   *bytes = num_blocks * num_kv_heads * head_page_bytes(fmt, head_dim);
   return KVQ_OK;
 }
 
+kvq_status kv_pq3_codebook(float* cb) {
+  if (!cb) return fail(KVQ_ERR_INVALID_ARG, "cb is NULL");
+  // Lloyd's algorithm on the standard normal density: the thresholds are the
+  // midpoints of neighbouring centroids, each centroid the density's mean
+  // over its cell, iterated to a fixed point from evenly spaced centroids.
+  const double inv_sqrt2pi = 0.3989422804014327, inv_sqrt2 = 0.7071067811865476;
+  auto pdf = [&](double x) { return std::isinf(x) ? 0.0 : inv_sqrt2pi * std::exp(-0.5 * x * x); };
+  auto cdf = [&](double x) { return 0.5 * std::erfc(-x * inv_sqrt2); };
+  double c[8];
+  for (int k = 0; k < 8; ++k) c[k] = (k - 3.5) * 0.5;
+  for (int it = 0; it < 100000; ++it) {
+    double t[9];
+    t[0] = -INFINITY;
+    t[8] = INFINITY;
+    for (int k = 1; k < 8; ++k) t[k] = 0.5 * (c[k - 1] + c[k]);
+    double moved = 0.0;
+    for (int k = 0; k < 8; ++k) {
+      const double m = (pdf(t[k]) - pdf(t[k + 1])) / (cdf(t[k + 1]) - cdf(t[k]));
+      moved = std::fmax(moved, std::fabs(m - c[k]));
+      c[k] = m;
+    }
+    if (moved < 1e-15) break;
+  }
+  // scale to one coordinate of a unit vector in 128 dimensions, then round to
+  // the nearest f16 value (11 significant bits, ties to even)
+  for (int k = 0; k < 8; ++k) {
+    const double v = c[k] / std::sqrt(128.0);
+    int e = 0;
+    std::frexp(v, &e);
+    const double ulp = std::ldexp(1.0, e - 11);
+    cb[k] = static_cast<float>(std::nearbyint(v / ulp) * ulp);  // default rounding: to even
+  }
+  return KVQ_OK;
+}
+
 kvq_status kv_scale_from_absmax(int32_t fmt, float amax, float* scale) {
+  if (fmt == KVQ_FMT_PQ3)
+    return fail(KVQ_ERR_UNSUPPORTED, "PQ3 has no abs-max scale (see kv_pq3_codebook)");
   if (fmt < 0 || fmt > 2) return fail(KVQ_ERR_UNSUPPORTED, "unknown format %d", fmt);
   if (!scale) return fail(KVQ_ERR_INVALID_ARG, "scale is NULL");
   if (!(amax >= 0.0f) || isinf(amax)) return fail(KVQ_ERR_INVALID_ARG, "amax must be finite, >= 0");
@@ -320,6 +370,8 @@ kvq_status kv_scale_from_absmax(int32_t fmt, float amax, float* scale) {
 
 kvq_status kv_scale_from_absmax_device(int32_t fmt, const float* d_amax, float* d_scale,
                                        kvq_stream stream) {
+  if (fmt == KVQ_FMT_PQ3)
+    return fail(KVQ_ERR_UNSUPPORTED, "PQ3 has no abs-max scale (see kv_pq3_codebook)");
   if (fmt < 0 || fmt > 2) return fail(KVQ_ERR_UNSUPPORTED, "unknown format %d", fmt);
   if (!d_amax || !d_scale) return fail(KVQ_ERR_INVALID_ARG, "d_amax/d_scale is NULL");
   kvq_status s = check_device();
@@ -480,6 +532,8 @@ kvq_status decode_impl(int32_t fmt, const void* q, const kvq_cache* cache,
   p.v_scale = d_v_scale;
   p.q_scale = d_q_scale;
   p.prob_scale = d_prob_scale;
+  p.kc = static_cast<const uint8_t*>(cache->k);
+  p.vc = static_cast<const uint8_t*>(cache->v);
   p.out = out;
   p.lse = lse;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
@@ -545,6 +599,7 @@ kvq_status kv_prefill_attention(int32_t fmt, const void* q, const kvq_cache* cac
                                 int32_t* d_err, kvq_stream stream) {
   kvq_status s = check_cache(fmt, cache);
   if (s != KVQ_OK) return s;
+  if (fmt == KVQ_FMT_PQ3) return fail(KVQ_ERR_UNSUPPORTED, "no chunked prefill for PQ3");
   const int D = cache->head_dim, Hkv = cache->num_kv_heads;
   if (num_seqs < 0 || num_q_tokens < 0)
     return fail(KVQ_ERR_INVALID_ARG, "num_seqs %d / num_q_tokens %d", num_seqs, num_q_tokens);

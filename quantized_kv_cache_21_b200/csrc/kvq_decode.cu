@@ -86,12 +86,13 @@ struct Fmt<1, 128> {
   __device__ static int v_elem(int gid, int i) { return 16 * gid + i; }
   __device__ static void issue(uint8_t* st, uint64_t* bar, const CUtensorMap* mk,
                                const CUtensorMap* mv, const CUtensorMap*, const CUtensorMap*,
-                               int h, int blk) {
+                               int h, int blk, const DecodeParams&) {
     mbar_arrive_expect_tx(bar, TX);
     tma_load_4d(st, mk, bar, 0, 0, h, blk);
     tma_load_4d(st + V_OFF, mv, bar, 0, 0, h, blk);
   }
-  __device__ static void prefetch(const CUtensorMap* mk, const CUtensorMap* mv, int h, int blk) {
+  __device__ static void prefetch(const CUtensorMap* mk, const CUtensorMap* mv, int h, int blk,
+                                  const DecodeParams&) {
     tma_prefetch_l2_4d(mk, 0, 0, h, blk);
     tma_prefetch_l2_4d(mv, 0, 0, h, blk);
   }
@@ -148,12 +149,13 @@ struct Fmt<1, 64> {
   __device__ static int v_elem(int gid, int i) { return 8 * gid + i; }
   __device__ static void issue(uint8_t* st, uint64_t* bar, const CUtensorMap* mk,
                                const CUtensorMap* mv, const CUtensorMap*, const CUtensorMap*,
-                               int h, int blk) {
+                               int h, int blk, const DecodeParams&) {
     mbar_arrive_expect_tx(bar, TX);
     tma_load_4d(st, mk, bar, 0, 0, h, blk);
     tma_load_4d(st + V_OFF, mv, bar, 0, 0, h, blk);
   }
-  __device__ static void prefetch(const CUtensorMap* mk, const CUtensorMap* mv, int h, int blk) {
+  __device__ static void prefetch(const CUtensorMap* mk, const CUtensorMap* mv, int h, int blk,
+                                  const DecodeParams&) {
     tma_prefetch_l2_4d(mk, 0, 0, h, blk);
     tma_prefetch_l2_4d(mv, 0, 0, h, blk);
   }
@@ -204,12 +206,13 @@ struct Fmt<0, 64> {
   __device__ static int v_elem(int gid, int i) { return 8 * gid + i; }
   __device__ static void issue(uint8_t* st, uint64_t* bar, const CUtensorMap* mk,
                                const CUtensorMap* mv, const CUtensorMap*, const CUtensorMap*,
-                               int h, int blk) {
+                               int h, int blk, const DecodeParams&) {
     mbar_arrive_expect_tx(bar, TX);
     tma_load_4d(st, mk, bar, 0, 0, h, blk);
     tma_load_4d(st + V_OFF, mv, bar, 0, 0, h, blk);
   }
-  __device__ static void prefetch(const CUtensorMap* mk, const CUtensorMap* mv, int h, int blk) {
+  __device__ static void prefetch(const CUtensorMap* mk, const CUtensorMap* mv, int h, int blk,
+                                  const DecodeParams&) {
     tma_prefetch_l2_4d(mk, 0, 0, h, blk);
     tma_prefetch_l2_4d(mv, 0, 0, h, blk);
   }
@@ -271,14 +274,15 @@ struct Fmt<0, 128> {
   }
   __device__ static void issue(uint8_t* st, uint64_t* bar, const CUtensorMap* mk,
                                const CUtensorMap* mv, const CUtensorMap*, const CUtensorMap*,
-                               int h, int blk) {
+                               int h, int blk, const DecodeParams&) {
     mbar_arrive_expect_tx(bar, TX);
     tma_load_4d(st, mk, bar, 0, 0, h, blk);
     tma_load_4d(st + 2048, mk, bar, 64, 0, h, blk);
     tma_load_4d(st + V_OFF, mv, bar, 0, 0, h, blk);
     tma_load_4d(st + V_OFF + 2048, mv, bar, 64, 0, h, blk);
   }
-  __device__ static void prefetch(const CUtensorMap* mk, const CUtensorMap* mv, int h, int blk) {
+  __device__ static void prefetch(const CUtensorMap* mk, const CUtensorMap* mv, int h, int blk,
+                                  const DecodeParams&) {
     tma_prefetch_l2_4d(mk, 0, 0, h, blk);
     tma_prefetch_l2_4d(mk, 64, 0, h, blk);
     tma_prefetch_l2_4d(mv, 0, 0, h, blk);
@@ -369,12 +373,13 @@ struct Fmt<2, 64> {
   __device__ static int v_elem(int gid, int i) { return 8 * gid + i; }
   __device__ static void issue(uint8_t* st, uint64_t* bar, const CUtensorMap* mk,
                                const CUtensorMap* mv, const CUtensorMap*, const CUtensorMap*,
-                               int h, int blk) {
+                               int h, int blk, const DecodeParams&) {
     mbar_arrive_expect_tx(bar, TX);
     tma_load_4d(st, mk, bar, 0, 0, h, blk);
     tma_load_4d(st + V_OFF, mv, bar, 0, 0, h, blk);
   }
-  __device__ static void prefetch(const CUtensorMap* mk, const CUtensorMap* mv, int h, int blk) {
+  __device__ static void prefetch(const CUtensorMap* mk, const CUtensorMap* mv, int h, int blk,
+                                  const DecodeParams&) {
     tma_prefetch_l2_4d(mk, 0, 0, h, blk);
     tma_prefetch_l2_4d(mv, 0, 0, h, blk);
   }
@@ -455,12 +460,13 @@ struct Fmt<2, 128> {
   __device__ static int v_elem(int gid, int i) { return 16 * gid + i; }
   __device__ static void issue(uint8_t* st, uint64_t* bar, const CUtensorMap* mk,
                                const CUtensorMap* mv, const CUtensorMap*, const CUtensorMap*,
-                               int h, int blk) {
+                               int h, int blk, const DecodeParams&) {
     mbar_arrive_expect_tx(bar, TX);
     tma_load_4d(st, mk, bar, 0, 0, h, blk);
     tma_load_4d(st + V_OFF, mv, bar, 0, 0, h, blk);
   }
-  __device__ static void prefetch(const CUtensorMap* mk, const CUtensorMap* mv, int h, int blk) {
+  __device__ static void prefetch(const CUtensorMap* mk, const CUtensorMap* mv, int h, int blk,
+                                  const DecodeParams&) {
     tma_prefetch_l2_4d(mk, 0, 0, h, blk);
     tma_prefetch_l2_4d(mv, 0, 0, h, blk);
   }
@@ -542,6 +548,113 @@ struct Fmt<2, 128> {
   }
 };
 
+// ---- PQ3 (3-bit planar-rotation codec of 128-element vectors), head_dim 128:
+// a head page is 16 fp32 norms and 16 rows of 48 index bytes (832 B; index i
+// of a row in bits [3i, 3i+3)), fetched whole by bulk copies, K's page then
+// V's.  Indices become exact f16 codebook values by two byte permutes over
+// the codebook's low and high bytes (tl, th), four values at a time.
+template <>
+struct Fmt<3, 128> {
+  static constexpr bool kBF16 = false;
+  static constexpr int STAGE = 1664, TX = 1664, V_OFF = 832, PAGE = 832;
+  static constexpr bool kLateV = false;
+  __device__ static int k_elem(int tig, int i) { return 32 * tig + i; }
+  __device__ static int v_elem(int gid, int i) { return 16 * gid + i; }
+  __device__ static const uint8_t* page(const uint8_t* base, const DecodeParams& p, int h,
+                                        int blk) {
+    return base + (static_cast<size_t>(blk) * p.Hkv + h) * PAGE;
+  }
+  __device__ static void issue(uint8_t* st, uint64_t* bar, const CUtensorMap*, const CUtensorMap*,
+                               const CUtensorMap*, const CUtensorMap*, int h, int blk,
+                               const DecodeParams& p) {
+    mbar_arrive_expect_tx(bar, TX);
+    bulk_load(st, page(p.kc, p, h, blk), PAGE, bar);
+    bulk_load(st + V_OFF, page(p.vc, p, h, blk), PAGE, bar);
+  }
+  __device__ static void prefetch(const CUtensorMap*, const CUtensorMap*, int h, int blk,
+                                  const DecodeParams& p) {
+    bulk_prefetch_l2(page(p.kc, p, h, blk), PAGE);
+    bulk_prefetch_l2(page(p.vc, p, h, blk), PAGE);
+  }
+  // Raw stage words: K rows gid, gid+8, their norms and the 12 index bytes of
+  // head-dim elements 32tig .. 32tig+31; V rows 2tig, 2tig+1, 2tig+8, 2tig+9,
+  // the 8 aligned bytes holding the indices of elements 16gid .. 16gid+15
+  // (bits [48 gid, 48 gid + 48) of the row), and the V norms of tokens gid and
+  // gid+8 (the token rows of P).
+  struct Raw {
+    uint32_t kw[2][3], vw[4][2];
+    float nk[2], nv[2];
+  };
+  __device__ static void load_raw_k(const uint8_t* st, int gid, int tig, Raw& r) {
+#pragma unroll
+    for (int rr = 0; rr < 2; ++rr) {
+      const int row = gid + 8 * rr;
+      const uint32_t* w = reinterpret_cast<const uint32_t*>(st + 64 + 48 * row + 12 * tig);
+      r.kw[rr][0] = w[0];
+      r.kw[rr][1] = w[1];
+      r.kw[rr][2] = w[2];
+      r.nk[rr] = reinterpret_cast<const float*>(st)[row];
+    }
+  }
+  __device__ static void load_raw_v(const uint8_t* st, int gid, int tig, Raw& r) {
+    const uint8_t* sv = st + V_OFF;
+    const int base = (6 * gid) & ~3;
+    const int rows[4] = {2 * tig, 2 * tig + 1, 2 * tig + 8, 2 * tig + 9};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t* w = reinterpret_cast<const uint32_t*>(sv + 64 + 48 * rows[i] + base);
+      r.vw[i][0] = w[0];
+      r.vw[i][1] = w[1];
+    }
+    r.nv[0] = reinterpret_cast<const float*>(sv)[gid];
+    r.nv[1] = reinterpret_cast<const float*>(sv)[gid + 8];
+  }
+  // f16x2 (c[i0], c[i1]) and (c[i2], c[i3]) of four 3-bit indices.
+  __device__ static void lookup4(uint32_t i0, uint32_t i1, uint32_t i2, uint32_t i3,
+                                 const uint32_t tl[2], const uint32_t th[2], uint32_t& p01,
+                                 uint32_t& p23) {
+    const uint32_t sel = i0 | (i1 << 4) | (i2 << 8) | (i3 << 12);
+    const uint32_t lo = prmt(tl[0], tl[1], sel), hi = prmt(th[0], th[1], sel);
+    p01 = prmt(lo, hi, 0x5140);
+    p23 = prmt(lo, hi, 0x7362);
+  }
+  // A fragments of QK: k-step s takes the 12-bit field at bit 12s of the
+  // thread's 96-bit run (elements 32tig + 4s .. +3).
+  __device__ static void conv_k(const Raw& r, uint32_t ka[8][4], const uint32_t tl[2],
+                                const uint32_t th[2]) {
+#pragma unroll
+    for (int s = 0; s < 8; ++s) {
+#pragma unroll
+      for (int rr = 0; rr < 2; ++rr) {
+        const int b = 12 * s, wi = b >> 5, sh = b & 31;
+        const uint32_t f =
+            (sh + 12 <= 32 ? (r.kw[rr][wi] >> sh) : __funnelshift_r(r.kw[rr][wi], r.kw[rr][wi + 1], sh)) &
+            0xFFFu;
+        lookup4(f & 7u, (f >> 3) & 7u, (f >> 6) & 7u, (f >> 9) & 7u, tl, th, ka[s][rr],
+                ka[s][2 + rr]);
+      }
+    }
+  }
+  // A fragments of PV: m-tile jj takes head-dim elements 16gid + 2jj, +1 of
+  // tokens 2tig, 2tig+1 (va[jj][0], [1]) and 2tig+8, 2tig+9 (va[jj][2], [3]).
+  __device__ static void conv_v(const Raw& r, uint32_t va[8][4], const uint32_t tl[2],
+                                const uint32_t th[2], int gid) {
+    const int sh0 = ((6 * gid) & 3) * 8;  // the run starts 0 or 16 bits into the words
+    uint64_t run[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      run[i] = ((static_cast<uint64_t>(r.vw[i][1]) << 32) | r.vw[i][0]) >> sh0;
+#pragma unroll
+    for (int jj = 0; jj < 8; ++jj) {
+      uint32_t f[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) f[i] = static_cast<uint32_t>(run[i] >> (6 * jj)) & 63u;
+      lookup4(f[0] & 7u, f[1] & 7u, f[0] >> 3, f[1] >> 3, tl, th, va[jj][0], va[jj][1]);
+      lookup4(f[2] & 7u, f[3] & 7u, f[2] >> 3, f[3] >> 3, tl, th, va[jj][2], va[jj][3]);
+    }
+  }
+};
+
 // Kernel shape per format: warps per CTA (NW, one CTA per SM) and ring stages
 // per warp (NSW).  Each warp owns NSW stages (~150-170 KB of ring per SM in
 // all) and refills a stage only after consuming it, so every mbarrier wait is
@@ -550,9 +663,9 @@ struct Fmt<2, 128> {
 // instruction latency, so those kernels run 16 warps (128 registers each).
 template <int FMT, int D>
 struct Shape {
-  static constexpr int NW = (FMT != 0 && D == 64) ? 16 : (FMT == 0 && D == 128) ? 10 : 12;
+  static constexpr int NW = (FMT != 0 && D == 64) ? 16 : ((FMT == 0 || FMT == 3) && D == 128) ? 10 : 12;
   static constexpr int STAGE = Fmt<FMT, D>::STAGE;
-  static constexpr int NSW = (FMT == 2 && D == 64) ? 7 : (FMT == 1 && D == 64) ? 5
+  static constexpr int NSW = (FMT == 2 && D == 64) ? 7 : (FMT == 1 && D == 64) ? 5 : FMT == 3 ? 6
                              : STAGE <= 2048 ? 6 : STAGE <= 3072 ? 4 : STAGE <= 4096 ? 3 : 2;
   static constexpr int WPART = 16 + 8 * D;  // floats of one partial: m[8], l[8], o[8][D]
 };
@@ -657,7 +770,7 @@ __device__ __forceinline__ void item_block(const DecodeParams& p, const UnitTabl
 // c_first + n)) into out / lse; threads t of nthreads share the float4
 // columns.  Partials are read kBatch at a time, all loads of a batch in
 // flight together (one pass when n <= kBatch), folded with a running max.
-template <int D, int WPART>
+template <int D, int WPART, bool kRot>
 __device__ __forceinline__ void final_merge(const DecodeParams& p, int u, int b, int h, int grp,
                                             int c_first, int n, float vs, int t, int nthreads) {
   const float kInf = __int_as_float(0x7f800000);
@@ -708,6 +821,12 @@ __device__ __forceinline__ void final_merge(const DecodeParams& p, int u, int b,
     }
     const float sc = L > 0.f ? vs / L : 0.f;
     const size_t row = static_cast<size_t>(b) * p.Hq + h * p.G + qi;
+    if constexpr (kRot) {  // PQ3: rotate the pairs (d4, d4+1), (d4+2, d4+3) back
+      const float c0 = __ldg(p.v_scale + 8 + d4), s0 = __ldg(p.v_scale + 9 + d4);
+      const float c1 = __ldg(p.v_scale + 10 + d4), s1 = __ldg(p.v_scale + 11 + d4);
+      acc = make_float4(fmaf(c0, acc.x, s0 * acc.y), fmaf(c0, acc.y, -(s0 * acc.x)),
+                        fmaf(c1, acc.z, s1 * acc.w), fmaf(c1, acc.w, -(s1 * acc.z)));
+    }
     *reinterpret_cast<float4*>(p.out + row * D + d4) =
         make_float4(acc.x * sc, acc.y * sc, acc.z * sc, acc.w * sc);
     if (d4 == 0 && p.lse) p.lse[row] = L > 0.f ? (M + log2f(L) - kPLog2) * kLn2 : -kInf;
@@ -762,13 +881,37 @@ __global__ void __launch_bounds__(Shape<FMT, D>::NW * 32, 1)
   // Scales: FP8 needs s > 0, NVFP4 g >= 0 (0 = an all-zero tensor); both finite.
   float ks = 1.f, vs = 1.f;
   bool scale_ok = true;
-  if constexpr (FMT != 0) {
+  // PQ3: the K and V codebooks (the parameter blocks' first 8 values, f16
+  // values by contract) as byte tables for the index lookups, and the
+  // check that each is finite and ascending
+  uint32_t tkl[2] = {0u, 0u}, tkh[2] = {0u, 0u}, tvl[2] = {0u, 0u}, tvh[2] = {0u, 0u};
+  if constexpr (FMT == 1 || FMT == 2) {
     ks = __ldg(p.k_scale);
     vs = __ldg(p.v_scale);
     if (FMT == 1)
       scale_ok = ks > 0.f && vs > 0.f && ks < kInf && vs < kInf;
     else
       scale_ok = ks >= 0.f && vs >= 0.f && ks < kInf && vs < kInf;
+    if (!scale_ok && c == 0 && tid == 0) set_err(p.d_err, kErrScale);
+  } else if constexpr (FMT == 3) {
+#pragma unroll
+    for (int kv = 0; kv < 2; ++kv) {
+      const float* cb = kv ? p.v_scale : p.k_scale;
+      float v[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) v[k] = __ldg(cb + k);
+#pragma unroll
+      for (int k = 0; k < 7; ++k) scale_ok = scale_ok && v[k] < v[k + 1];
+      scale_ok = scale_ok && v[0] > -kInf && v[7] < kInf;
+      const uint32_t w01 = pack_f16x2(v[0], v[1]), w23 = pack_f16x2(v[2], v[3]);
+      const uint32_t w45 = pack_f16x2(v[4], v[5]), w67 = pack_f16x2(v[6], v[7]);
+      uint32_t* tl = kv ? tvl : tkl;
+      uint32_t* th = kv ? tvh : tkh;
+      tl[0] = prmt(w01, w23, 0x6420);  // low bytes of c0 .. c3
+      tl[1] = prmt(w45, w67, 0x6420);
+      th[0] = prmt(w01, w23, 0x7531);  // high bytes
+      th[1] = prmt(w45, w67, 0x7531);
+    }
     if (!scale_ok && c == 0 && tid == 0) set_err(p.d_err, kErrScale);
   }
   // FP8 attention: the E4M3 scales of q and P (both > 0 and finite).  The
@@ -798,10 +941,28 @@ __global__ void __launch_bounds__(Shape<FMT, D>::NW * 32, 1)
   // Query fragments (B operand of QK) of unit u; padded heads are 0.  The
   // thread's head-dim elements come in 16-byte runs of 8.
   uint32_t qb[KS][2];
+  // PQ3: the scores are q . (|k| R^T c[idx]) = |k| (R q) . c[idx]: q is rotated
+  // once, q' = R q (fp32), and enters QK as a 16-bit high part (qb) and its
+  // residual (qbl), so the product keeps ~22 bits of q'
+  uint32_t qbl[FMT == 3 ? KS : 1][2];
   // FP8 attention: the E4M3 query as the A operand of QK (rows = heads, row
   // gid; the padding rows gid+8 are zero): per 32-element k-step s, a0 holds
   // head-dim elements k_elem(tig, 8s .. 8s+3) and a2 elements 8s+4 .. 8s+7.
   uint32_t qa[QP ? D / 32 : 1][2];
+  // Format-specific decode of a stage's words into MMA fragments (PQ3 also
+  // needs its codebook tables).
+  auto conv_k_any = [&](const typename F::Raw& raw, uint32_t ka[KS][4]) {
+    if constexpr (FMT == 3)
+      F::conv_k(raw, ka, tkl, tkh);
+    else
+      F::conv_k(raw, ka);
+  };
+  auto conv_v_any = [&](const typename F::Raw& raw, uint32_t va[MT][4]) {
+    if constexpr (FMT == 3)
+      F::conv_v(raw, va, tvl, tvh, gid);
+    else
+      F::conv_v(raw, va);
+  };
   auto load_q = [&](int u) {
     const int grp = u % p.n_groups, h = (u / p.n_groups) % p.Hkv, b = u / (p.n_groups * p.Hkv);
     const int qi = grp * 8 + gid;
@@ -821,6 +982,26 @@ __global__ void __launch_bounds__(Shape<FMT, D>::NW * 32, 1)
           e[x] = f32x2_to_e4m3x2(__fdiv_rn(bf16_lo(ws[x]), qs), __fdiv_rn(bf16_hi(ws[x]), qs));
         qa[s][0] = (e[0] | (e[1] << 16)) ^ q_sign;
         qa[s][1] = (e[2] | (e[3] << 16)) ^ q_sign;
+      }
+    } else if constexpr (FMT == 3) {
+      const float* rot = p.k_scale + 8;
+#pragma unroll
+      for (int i = 0; i < D / 4; i += 8) {
+        const uint4 w = hv ? __ldg(reinterpret_cast<const uint4*>(qrow + F::k_elem(tig, i)))
+                           : make_uint4(0u, 0u, 0u, 0u);
+        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int x = 0; x < 4; ++x) {  // the pair of head-dim elements 2j, 2j+1
+          const int j = F::k_elem(tig, i) / 2 + x;
+          const float cs = __ldg(rot + 2 * j), sn = __ldg(rot + 2 * j + 1);
+          const float a = bf16_lo(ws[x]), b = bf16_hi(ws[x]);
+          const float y0 = fmaf(cs, a, -(sn * b)), y1 = fmaf(sn, a, cs * b);
+          const uint32_t hi = pack_f16x2(y0, y1);
+          float h0, h1;
+          unpack_f16x2(hi, h0, h1);
+          qb[i / 4 + x / 2][x & 1] = hi ^ q_sign;
+          qbl[i / 4 + x / 2][x & 1] = pack_f16x2(y0 - h0, y1 - h1) ^ q_sign;
+        }
       }
     } else {
 #pragma unroll
@@ -887,7 +1068,7 @@ __global__ void __launch_bounds__(Shape<FMT, D>::NW * 32, 1)
   // Ask L2 for the pages of this warp's first stages (the guessed block ids)
   // while the unit table is built; a wrong guess only costs a prefetch.
   if (p.window <= 0 && lane < NSW && spec0 >= 0 && spec0 < p.num_blocks)
-    F::prefetch(&mk, &mv, (u0 / p.n_groups) % p.Hkv, spec0);
+    F::prefetch(&mk, &mv, (u0 / p.n_groups) % p.Hkv, spec0, p);
   if (lane < NSW) mbar_init(&bars[lane], 1);  // each warp its own stages
   mbar_init_fence();
   __syncthreads();
@@ -942,7 +1123,7 @@ __global__ void __launch_bounds__(Shape<FMT, D>::NW * 32, 1)
       uint64_t* bar = &bars[stg];
       fence_proxy_async_smem();  // the warp's reads of this stage precede the copy
       if (ok) {
-        F::issue(ring + stg * F::STAGE, bar, &mk, &mv, &mks, &mvs, cur_h, cur_blk);
+        F::issue(ring + stg * F::STAGE, bar, &mk, &mv, &mks, &mvs, cur_h, cur_blk, p);
       } else {
         set_err(p.d_err, kErrBlockId);
         mbar_arrive(bar);  // completes the phase with no data; the page is skipped
@@ -957,7 +1138,7 @@ __global__ void __launch_bounds__(Shape<FMT, D>::NW * 32, 1)
     if (lane < n0) {
       uint64_t* bar = &bars[lane];
       if ((ok_win >> lane) & 1u) {
-        F::issue(ring + lane * F::STAGE, bar, &mk, &mv, &mks, &mvs, cur_h, cur_blk);
+        F::issue(ring + lane * F::STAGE, bar, &mk, &mv, &mks, &mvs, cur_h, cur_blk, p);
       } else {
         set_err(p.d_err, kErrBlockId);
         mbar_arrive(bar);  // completes the phase with no data; the page is skipped
@@ -997,7 +1178,7 @@ __global__ void __launch_bounds__(Shape<FMT, D>::NW * 32, 1)
       return;
     }
     uint32_t ka[KS][4];
-    F::conv_k(raw, ka);
+    conv_k_any(raw, ka);
     float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int s = 0; s < KS; ++s) {
@@ -1040,6 +1221,7 @@ __global__ void __launch_bounds__(Shape<FMT, D>::NW * 32, 1)
     float n0 = 1e30f, n1 = 1e30f;
     // FP8 attention: running reference max mq and normaliser lq of head gid
     float mq = -kInf, lq = 0.f;
+    int kb = 0;  // PQ3: exponent of the V-norm scale P carries (see below)
     float o[MT][4];
 #pragma unroll
     for (int jj = 0; jj < MT; ++jj) o[jj][0] = o[jj][1] = o[jj][2] = o[jj][3] = 0.f;
@@ -1166,7 +1348,7 @@ __global__ void __launch_bounds__(Shape<FMT, D>::NW * 32, 1)
           va[2 * k + 1][1] = prmt(xyh, zth, 0x7632);  // byte 3
         }
       } else {
-        F::conv_v(raw, va);
+        conv_v_any(raw, va);
       }
     };
     // Softmax of a page, part 2, and O^T += V^T P^T.  Tokens at or past
@@ -1302,13 +1484,17 @@ __global__ void __launch_bounds__(Shape<FMT, D>::NW * 32, 1)
         float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
         // ---- S^T = K Q^T on tensor cores (two accumulator chains)
         auto qk = [&]() {
-          F::conv_k(raw, ka);
+          conv_k_any(raw, ka);
   #pragma unroll
           for (int s = 0; s < KS; ++s) {
-            if (s & 1)
+            if constexpr (FMT == 3) {  // q' high part and residual, two chains
+              mma16816<false>(sa, ka[s], qb[s][0], qb[s][1]);
+              mma16816<false>(sb, ka[s], qbl[s][0], qbl[s][1]);
+            } else if (s & 1) {
               mma16816<F::kBF16>(sb, ka[s], qb[s][0], qb[s][1]);
-            else
+            } else {
               mma16816<F::kBF16>(sa, ka[s], qb[s][0], qb[s][1]);
+            }
           }
         };
         if constexpr (F::kLateV) {
@@ -1329,14 +1515,24 @@ __global__ void __launch_bounds__(Shape<FMT, D>::NW * 32, 1)
         }
         if (!valid) continue;
         if constexpr (!F::kLateV) qk();
-        F::conv_v(raw, va);
+        conv_v_any(raw, va);
 
         // raw scores r = q . k_code (the scale c_log2 is applied below)
         float r0 = sa[0] + sb[0], r1 = sa[1] + sb[1], r2 = sa[2] + sb[2], r3 = sa[3] + sb[3];
+        if constexpr (FMT == 3) {  // times the K norms of tokens gid, gid+8
+          r0 *= raw.nk[0];
+          r1 *= raw.nk[0];
+          r2 *= raw.nk[1];
+          r3 *= raw.nk[1];
+        }
         if (k == k_end - 1 && n_last < kPage) {  // last, partial page: mask tokens past the length
           const int n_valid = n_last;
           if (gid >= n_valid) r0 = r1 = -kInf;
           if (gid + 8 >= n_valid) r2 = r3 = -kInf;
+          if constexpr (FMT == 3) {  // unwritten norms may be NaN
+            if (gid >= n_valid) raw.nv[0] = 0.f;
+            if (gid + 8 >= n_valid) raw.nv[1] = 0.f;
+          }
           const uint32_t m01 = (2 * tig < n_valid ? 0x0000FFFFu : 0u) |
                                (2 * tig + 1 < n_valid ? 0xFFFF0000u : 0u);
           const uint32_t m23 = (2 * tig + 8 < n_valid ? 0x0000FFFFu : 0u) |
@@ -1389,9 +1585,37 @@ __global__ void __launch_bounds__(Shape<FMT, D>::NW * 32, 1)
           e2 = s2 + n0;
           e3 = s3 + n1;
         }
-        const float q0 = fast_exp2(e0), q1 = fast_exp2(e1), q2 = fast_exp2(e2), q3 = fast_exp2(e3);
+        float q0 = fast_exp2(e0), q1 = fast_exp2(e1), q2 = fast_exp2(e2), q3 = fast_exp2(e3);
         l0 += q0 + q2;  // l and O carry the factor 2^kPLog2, removed at normalisation
         l1 += q1 + q3;
+        if constexpr (FMT == 3) {
+          // P also carries the V norms of its tokens (gid, gid+8), over a
+          // warp-uniform power of two 2^(kb - 126) at or above every V norm of
+          // the segment so far (kb: the largest biased fp32 exponent), which
+          // keeps it below 2^15 in f16; O takes the factor back at the segment
+          // end, and is rescaled (exactly) when kb grows
+          const int e_0 = (__float_as_int(raw.nv[0]) >> 23) & 0xFF;
+          const int e_1 = (__float_as_int(raw.nv[1]) >> 23) & 0xFF;
+          const int ep = min(__reduce_max_sync(0xffffffffu, max(e_0, e_1)), 252);
+          if (ep > kb) {
+            const int dd = 127 + kb - ep;
+            const float a = dd >= 1 ? __int_as_float(dd << 23) : 0.f;
+#pragma unroll
+            for (int jj = 0; jj < MT; ++jj) {
+              o[jj][0] *= a;
+              o[jj][1] *= a;
+              o[jj][2] *= a;
+              o[jj][3] *= a;
+            }
+            kb = ep;
+          }
+          const float sc = __int_as_float((253 - kb) << 23);  // 2^(126 - kb)
+          const float g0 = raw.nv[0] * sc, g1 = raw.nv[1] * sc;
+          q0 *= g0;
+          q1 *= g0;
+          q2 *= g1;
+          q3 *= g1;
+        }
 
         // ---- P^T fragments: high part + residual, transposed in registers
         uint32_t x0h, x1h, x0l, x1l;
@@ -1424,6 +1648,16 @@ __global__ void __launch_bounds__(Shape<FMT, D>::NW * 32, 1)
     }
     k_base = k_end;
 
+    if constexpr (FMT == 3) {  // O back to absolute units: times 2^(kb - 126)
+      const float a = __int_as_float((kb + 1) << 23);
+#pragma unroll
+      for (int jj = 0; jj < MT; ++jj) {
+        o[jj][0] *= a;
+        o[jj][1] *= a;
+        o[jj][2] *= a;
+        o[jj][3] *= a;
+      }
+    }
     // ---- segment end: warp partials -> shared slots, merged by the CTA
     float* wp = slots + warp * S::WPART;  // m[8], l[8], o[8][D]
     if constexpr (QP) {  // head gid's sums are spread over the tig lanes
@@ -1474,6 +1708,38 @@ __global__ void __launch_bounds__(Shape<FMT, D>::NW * 32, 1)
     __syncthreads();
     const bool alone = c_first == c_last;
     float* gpart = p.ws_part + (static_cast<size_t>(u) + c) * S::WPART;
+    if constexpr (FMT == 3) {
+      // PQ3: O holds R_v (out); an output pair (2j, 2j+1) is rotated back,
+      // out_2j = cos_j a + sin_j b, out_2j+1 = cos_j b - sin_j a
+      for (int idx = tid; idx < 4 * D; idx += NT) {
+        const int hh = idx / (D / 2), d = 2 * (idx - hh * (D / 2));
+        const float M = s_ml[0][hh], L = s_ml[1][hh];
+        float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+        for (int w = 0; w < NW; ++w) {
+          a0 += s_wt[w][hh] * slots[w * S::WPART + 16 + hh * D + d];
+          a1 += s_wt[w][hh] * slots[w * S::WPART + 16 + hh * D + d + 1];
+        }
+        if (alone) {
+          const int qi = grp * 8 + hh;
+          if (qi < p.G) {
+            const size_t row = static_cast<size_t>(b) * p.Hq + h * p.G + qi;
+            const float cs = __ldg(p.v_scale + 8 + d), sn = __ldg(p.v_scale + 9 + d);
+            const float sc = L > 0.f ? vs_out / L : 0.f;
+            p.out[row * D + d] = fmaf(cs, a0, sn * a1) * sc;
+            p.out[row * D + d + 1] = fmaf(cs, a1, -(sn * a0)) * sc;
+            if (d == 0 && p.lse) p.lse[row] = L > 0.f ? (M + log2f(L) - kPLog2) * kLn2 : -kInf;
+          }
+        } else {
+          gpart[16 + hh * D + d] = a0;
+          gpart[16 + hh * D + d + 1] = a1;
+          if (d == 0) {
+            gpart[hh] = M;
+            gpart[8 + hh] = L;
+          }
+        }
+      }
+    } else
     for (int idx = tid; idx < 8 * D; idx += NT) {
       const int hh = idx / D, d = idx - hh * D;
       const float M = s_ml[0][hh], L = s_ml[1][hh];
@@ -1507,7 +1773,8 @@ __global__ void __launch_bounds__(Shape<FMT, D>::NW * 32, 1)
       }
       __syncthreads();
       if (s_last) {
-        final_merge<D, S::WPART>(p, u, b, h, grp, c_first, c_last - c_first + 1, vs_out, tid, NT);
+        final_merge<D, S::WPART, FMT == 3>(p, u, b, h, grp, c_first, c_last - c_first + 1, vs_out,
+                                           tid, NT);
         if (tid == 0) p.ws_cnt[u] = 0u;  // ready for the next launch
       }
     }
@@ -1566,6 +1833,7 @@ bool decode_config(int fmt, int D, DecodeConfig* cfg) {
     case 1128: config_t<1, 128>(cfg); return true;
     case 2064: config_t<2, 64>(cfg); return true;
     case 2128: config_t<2, 128>(cfg); return true;
+    case 3128: config_t<3, 128>(cfg); return true;
   }
   return false;
 }
@@ -1584,6 +1852,7 @@ cudaError_t launch_decode(int fmt, int D, const CUtensorMap* maps, const DecodeP
     case 1128: return launch_t<1, 128>(maps, p, ctas, stream);
     case 2064: return launch_t<2, 64>(maps, p, ctas, stream);
     case 2128: return launch_t<2, 128>(maps, p, ctas, stream);
+    case 3128: return launch_t<3, 128>(maps, p, ctas, stream);
   }
   return cudaErrorInvalidValue;
 }

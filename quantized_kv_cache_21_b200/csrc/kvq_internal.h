@@ -15,8 +15,10 @@ struct DecodeParams {
   const uint16_t* q;          // [B][Hq][D] bf16
   const int32_t* block_table; // [B][max_blocks]
   const int32_t* seq_lens;    // [B]
-  const float* k_scale;       // device scalar (FP8: s, NVFP4: g); unused for BF16
+  const float* k_scale;       // device scalar (FP8: s, NVFP4: g; PQ3: 136-float parameter block)
   const float* v_scale;
+  const uint8_t* kc;          // cache buffers (PQ3 pages are fetched by address)
+  const uint8_t* vc;
   const float* q_scale;       // FP8 attention only: device scalar, E4M3 scale of q
   const float* prob_scale;    // FP8 attention only: device scalar, E4M3 scale of P
   float* out;                 // [B][Hq][D]

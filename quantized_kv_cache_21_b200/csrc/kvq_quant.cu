@@ -295,6 +295,138 @@ __global__ void dequantize_kernel(int fmt, const uint8_t* kc, const uint8_t* vc,
   reinterpret_cast<float4*>(out)[1] = make_float4(v[4], v[5], v[6], v[7]);
 }
 
+// ------------------------------------------------------------------ PQ3
+// 3-bit planar-rotation codec of 128-element vectors ("AMD MI300X - KV Cache
+// Compression Benchmark", "Key Results": 52-byte blocks, 4.923x against FP16;
+// the planar rotation's 256 FMAs; a Lloyd-Max codebook).  Head page: 16 fp32
+// norms, then 16 rows of 48 bytes of 3-bit indices (index i in bits [3i,
+// 3i+3) of the row's little-endian bit string).  Parameter block of a tensor:
+// 8 ascending codebook values, then 64 (cos, sin) pairs.
+constexpr int kPq3Page = 832;
+
+// The codebook must be finite and ascending; anything else is a bad scale.
+__device__ __forceinline__ bool pq3_params_ok(const float* cb) {
+  bool ok = true;
+#pragma unroll
+  for (int k = 0; k < 7; ++k) ok = ok && cb[k] < cb[k + 1];
+  return ok && cb[0] > -kInf && cb[7] < kInf;
+}
+
+// One warp per (token, K|V, head) row; lane l holds elements 4l .. 4l+3.
+// Every fp32 step is the format's fixed one: the sum of squares as a
+// pairwise tree in index order (elements, then pairs, then the lanes'
+// butterfly), sqrt and division rounded to nearest, the rotation's explicit
+// roundings, and the index as the count of thresholds below y.
+__global__ void quantize_pq3_kernel(const QuantParams p) {
+  griddep_launch_dependents();  // a following decode may start its prologue
+  const int lane = threadIdx.x & 31;
+  const int64_t nwarps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  const int64_t rows = p.T * 2 * p.H;
+  for (int64_t r = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; r < rows;
+       r += nwarps) {
+    const int64_t t = r / (2 * p.H);
+    const int rem = static_cast<int>(r - t * 2 * p.H), kv = rem / p.H, h = rem - kv * p.H;
+    int64_t slot = -1;
+    if (lane == 0) slot = resolve_slot(p, t);  // errors reported once
+    slot = __shfl_sync(0xffffffffu, slot, 0);
+    if (slot < 0) continue;
+    const float* prm = kv ? p.v_scale : p.k_scale;
+    float cb[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) cb[k] = __ldg(prm + k);
+    if (!pq3_params_ok(cb)) {
+      if (lane == 0) set_err(p.d_err, kErrScale);
+      continue;
+    }
+    const uint16_t* x = (kv ? p.v : p.k) + (t * p.H + h) * 128;
+    const uint2 w = *reinterpret_cast<const uint2*>(x + 4 * lane);
+    const float x0 = bf16_lo(w.x), x1 = bf16_hi(w.x), x2 = bf16_lo(w.y), x3 = bf16_hi(w.y);
+    float ss = __fadd_rn(__fadd_rn(__fmul_rn(x0, x0), __fmul_rn(x1, x1)),
+                         __fadd_rn(__fmul_rn(x2, x2), __fmul_rn(x3, x3)));
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) ss = __fadd_rn(ss, __shfl_xor_sync(0xffffffffu, ss, off));
+    const float nrm = __fsqrt_rn(ss);
+    uint32_t code = 0;  // this lane's 4 indices, 3 bits each
+    if (nrm != 0.f) {
+      const float u[4] = {__fdiv_rn(x0, nrm), __fdiv_rn(x1, nrm), __fdiv_rn(x2, nrm),
+                          __fdiv_rn(x3, nrm)};
+      float thr[7];
+#pragma unroll
+      for (int k = 0; k < 7; ++k) thr[k] = __fmul_rn(__fadd_rn(cb[k], cb[k + 1]), 0.5f);
+#pragma unroll
+      for (int pr = 0; pr < 2; ++pr) {  // pairs j = 2 lane + pr: elements 2j, 2j+1
+        const int j = 2 * lane + pr;
+        const float c = __ldg(prm + 8 + 2 * j), sn = __ldg(prm + 9 + 2 * j);
+        const float u0 = u[2 * pr], u1 = u[2 * pr + 1];
+        const float y[2] = {__fmaf_rn(c, u0, -__fmul_rn(sn, u1)),
+                            __fmaf_rn(sn, u0, __fmul_rn(c, u1))};
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          uint32_t k = 0;
+#pragma unroll
+          for (int q = 0; q < 7; ++q) k += y[e] > thr[q] ? 1u : 0u;
+          code |= k << (3 * (2 * pr + e));
+        }
+      }
+    }
+    // 32-bit word wd (lanes 0..11) of the row gathers the 12-bit chunks of
+    // lanes 32 wd / 12 .. (32 wd + 31) / 12
+    const int wd = lane < 12 ? lane : 11;
+    const int a = (32 * wd) / 12, b = (32 * wd + 31) / 12;
+    uint32_t word = 0;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int l = min(a + q, 31);
+      const uint32_t v = __shfl_sync(0xffffffffu, code, l);
+      const int sh = 12 * (a + q) - 32 * wd;
+      if (a + q <= b) word |= sh >= 0 ? v << sh : v >> (-sh);
+    }
+    uint8_t* page = (kv ? p.vc : p.kc) +
+                    ((slot / kPage) * p.H + h) * static_cast<int64_t>(kPq3Page);
+    const int o = static_cast<int>(slot % kPage);
+    if (lane < 12) *reinterpret_cast<uint32_t*>(page + 64 + 48 * o + 4 * lane) = word;
+    if (lane == 0) *reinterpret_cast<float*>(page + 4 * o) = nrm;
+  }
+}
+
+// The dequantised fp32 row of a PQ3 slot: x_hat_2j = nrm * fma(cos, Y0, sin *
+// Y1), x_hat_2j+1 = nrm * fma(cos, Y1, -(sin * Y0)).  One warp per (slot, K|V,
+// head) row, lane l writing elements 4l .. 4l+3.
+__global__ void dequantize_pq3_kernel(const uint8_t* kc, const uint8_t* vc, int64_t num_blocks,
+                                      int H, const int64_t* slots, int64_t n, const float* ks,
+                                      const float* vs, float* ko, float* vo, int* d_err) {
+  const int lane = threadIdx.x & 31;
+  const int64_t r = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  if (r >= n * 2 * H) return;
+  const int h = static_cast<int>(r % H), kv = static_cast<int>((r / H) & 1);
+  const int64_t i = r / (2 * H);
+  const int64_t slot = __ldg(slots + i);
+  if (slot < 0 || slot / kPage >= num_blocks) {
+    if (lane == 0 && h == 0 && kv == 0) set_err(d_err, kErrSlot);
+    return;
+  }
+  const float* prm = kv ? vs : ks;
+  const uint8_t* page = (kv ? vc : kc) + ((slot / kPage) * H + h) * static_cast<int64_t>(kPq3Page);
+  const int o = static_cast<int>(slot % kPage);
+  const float nrm = *reinterpret_cast<const float*>(page + 4 * o);
+  const uint32_t* row = reinterpret_cast<const uint32_t*>(page + 64 + 48 * o);
+  const int bit = 12 * lane, wi = bit >> 5, sh = bit & 31;
+  const uint32_t lo = row[wi], hi = wi < 11 ? row[wi + 1] : 0u;
+  const uint32_t code = __funnelshift_r(lo, hi, sh) & 0xFFFu;
+  float v[4];
+#pragma unroll
+  for (int pr = 0; pr < 2; ++pr) {
+    const int j = 2 * lane + pr;
+    const float c = __ldg(prm + 8 + 2 * j), sn = __ldg(prm + 9 + 2 * j);
+    const float y0 = __ldg(prm + ((code >> (6 * pr)) & 7u));
+    const float y1 = __ldg(prm + ((code >> (6 * pr + 3)) & 7u));
+    v[2 * pr] = __fmul_rn(nrm, __fmaf_rn(c, y0, __fmul_rn(sn, y1)));
+    v[2 * pr + 1] = __fmul_rn(nrm, __fmaf_rn(c, y1, -__fmul_rn(sn, y0)));
+  }
+  float* out = (kv ? vo : ko) + (i * H + h) * 128 + 4 * lane;
+  *reinterpret_cast<float4*>(out) = make_float4(v[0], v[1], v[2], v[3]);
+}
+
 // Per-16-bit-lane max of the magnitude bits of 8 BF16 values.
 __device__ __forceinline__ uint32_t absmax8(const uint4 a) {
   const uint32_t k = 0x7FFF7FFFu;
@@ -362,7 +494,12 @@ cudaError_t launch_quantize(int fmt, const QuantParams& p, cudaStream_t stream) 
   while (tpb < kTokPerBlock && p.T / (2 * tpb) >= 4 * static_cast<int64_t>(num_sms())) tpb *= 2;
   const int64_t blocks = (p.T + tpb - 1) / tpb;
   const unsigned grid = static_cast<unsigned>(blocks < (1 << 20) ? blocks : (1 << 20));
-  if (fmt == 1) {
+  if (fmt == 3) {  // one warp per row
+    const int64_t rows = p.T * 2 * p.H;
+    const int64_t cap = static_cast<int64_t>(num_sms()) * 16;
+    const int64_t b = (rows + 7) / 8;
+    quantize_pq3_kernel<<<static_cast<unsigned>(b < cap ? b : cap), threads, 0, stream>>>(p);
+  } else if (fmt == 1) {
     quantize_fp8_kernel<<<grid, threads, 0, stream>>>(p, tpb);
   } else if (fmt == 2) {
     quantize_nvfp4_kernel<<<grid, threads, 0, stream>>>(p, tpb);
@@ -378,6 +515,11 @@ cudaError_t launch_dequantize(int fmt, const uint8_t* kc, const uint8_t* vc, int
                               cudaStream_t stream) {
   if (n == 0) return cudaSuccess;
   const int threads = 256;
+  if (fmt == 3) {
+    dequantize_pq3_kernel<<<grid_for(n * 2 * H * 32, threads), threads, 0, stream>>>(
+        kc, vc, num_blocks, H, slots, n, ks, vs, ko, vo, d_err);
+    return cudaGetLastError();
+  }
   dequantize_kernel<<<grid_for(n * 2 * H * (D / 8), threads), threads, 0, stream>>>(
       fmt, kc, vc, num_blocks, H, D, slots, n, ks, vs, ko, vo, d_err);
   return cudaGetLastError();

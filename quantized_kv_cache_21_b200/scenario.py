@@ -15,12 +15,13 @@ import torch
 import quantized_kv_cache_21_b200 as kvq
 from quantized_kv_cache_21_b200 import workloads as wl
 
-BYTES_PER_ELEM = {"bf16": 2.0, "fp8": 1.0, "nvfp4": 4.5 / 8}
+BYTES_PER_ELEM = {"bf16": 2.0, "fp8": 1.0, "nvfp4": 4.5 / 8, "pq3": 52 / 128}
 
 
 def kv_scan_bytes(fmt: str, lens, H: int, D: int) -> int:
     """Algorithmic bytes one decode step must read from the cache: every
-    cached token's K and V for every KV head (NVFP4 block scales included)."""
+    cached token's K and V for every KV head (NVFP4 block scales and PQ3
+    norms included: 52 bytes per 128-element PQ3 vector)."""
     return int(round(sum(int(n) for n in lens) * H * 2 * D * BYTES_PER_ELEM[fmt]))
 
 
@@ -74,7 +75,11 @@ class DecodeScenario:
         self.d_ks, self.d_vs = self.scales[0:1], self.scales[1:2]
 
         # calibration: the first calib_tokens tokens of sequence 0, or all tokens
-        if self.fmt != "bf16":
+        # (PQ3 instead takes its codebook and a seeded planar rotation per tensor)
+        if self.fmt == "pq3":
+            self.d_ks = kvq.pq3_params(wl.planar_rotation(wl.rng_for(w.seed, 2)), dev)
+            self.d_vs = kvq.pq3_params(wl.planar_rotation(wl.rng_for(w.seed, 3)), dev)
+        elif self.fmt != "bf16":
             for b in range(B if w.calib_tokens is None else 1):
                 k, v = self.tokens(b)
                 n = int(self.lens[b]) if w.calib_tokens is None else w.calib_tokens

@@ -126,3 +126,17 @@ def test_header_is_plain_c99_and_links(L, tmp_path):
     assert out[0] == "0" and out[2] == "0"
     assert float.fromhex(out[1]) == float(np.float32(oracle.fp8_scale(448.0)))
     assert int(out[3]) == 37 * 3 * oracle.head_page_bytes("nvfp4", 128)
+
+
+def test_pq3_codebook_matches_the_oracle(L):
+    """The library's own Lloyd-Max solver gives the oracle's codebook, bit for
+    bit (8 ascending f16-representable values)."""
+    import numpy as np
+    cb = np.array(kvq.kv_pq3_codebook(), np.float32)
+    assert np.array_equal(cb, oracle.pq3_codebook())
+    assert np.array_equal(cb, cb.astype(np.float16).astype(np.float32))
+    with pytest.raises(kvq.KvqError, match="PQ3"):
+        kvq.kv_scale_from_absmax("pq3", 1.0)
+    assert kvq.kv_cache_bytes("pq3", 3, 2, 128) == 3 * 2 * 832
+    with pytest.raises(kvq.KvqError, match="head_dim 128"):
+        kvq.kv_cache_bytes("pq3", 3, 2, 64)

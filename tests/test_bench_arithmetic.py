@@ -27,9 +27,9 @@ def test_prefill_flops_of_the_benchmark_step():
 
 
 def test_kv_scan_bytes_brute_force():
-    H, D = 3, 64
+    H, D = 3, 128
     lens = np.array([17, 0, 100])
-    per_elem = {"bf16": 2.0, "fp8": 1.0, "nvfp4": 0.5 + 1 / 16}
+    per_elem = {"bf16": 2.0, "fp8": 1.0, "nvfp4": 0.5 + 1 / 16, "pq3": (4 + 48) / 128}
     for fmt, b in per_elem.items():
         elems = sum(int(n) for n in lens) * H * D * 2  # K and V
         assert kv_scan_bytes(fmt, lens, H, D) == round(elems * b)
