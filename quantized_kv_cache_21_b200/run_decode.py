@@ -24,7 +24,7 @@ from .scenario import DecodeScenario
 def main(argv=None) -> int:
     ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
     ap.add_argument("--workload", default="fp8-paged-4x32k", choices=sorted(wl.WORKLOADS))
-    ap.add_argument("--fmt", choices=["bf16", "fp8", "nvfp4"], default=None)
+    ap.add_argument("--fmt", choices=["bf16", "fp8", "nvfp4", "pq3"], default=None)
     ap.add_argument("--seq-len", type=int, default=None)
     ap.add_argument("--batch", type=int, default=None)
     ap.add_argument("--head-dim", type=int, choices=[64, 128], default=None)
