@@ -230,6 +230,22 @@ def test_variable_lengths_like_the_sweep(fmt, D):
 
 @pytest.mark.parametrize("fmt", FMTS)
 @pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("max_len", [16, 100, 700])
+def test_many_units_per_cta(fmt, D, max_len):
+    """Many short sequences (80 (sequence, KV head) units, lengths uniform in
+    [0, max_len]): the automatic split gives each CTA up to 27 units, taken
+    in turn, with some units spanning two CTAs and some empty, so the
+    per-unit merges inside a CTA meet the cross-CTA ones."""
+    rng = wl.rng_for(5200 + D + max_len, 3)
+    lens = rng.integers(0, max_len + 1, size=40).tolist()
+    c = Case(fmt, 40, 2, 16, D, lens, seed=5300 + D + max_len, factor=16.0)
+    out, lse = c.decode()
+    assert int(c.err.item()) == 0
+    assert_attention_close(out, lse, *c.reference())
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+@pytest.mark.parametrize("D", [64, 128])
 def test_decode_launched_right_after_a_write(fmt, D):
     """The decode may begin while a kv_quantize_write just before it on the
     stream is finishing: the last 1,200 tokens of every sequence are written

@@ -17,6 +17,7 @@ import torch
 
 import oracle
 import quantized_kv_cache_21_b200 as kvq
+from quantized_kv_cache_21_b200 import workloads as wl
 
 from gpu_common import DEV, LSE_RTOL, OUT_ATOL, Case, dev_scalar, new_err
 
@@ -94,6 +95,18 @@ def test_long_context_many_splits():
     assert np.abs(outs[0] - outs[2]).max() < 1e-4
 
 
+@pytest.mark.parametrize("max_len", [16, 100, 700])
+def test_many_units_per_cta(max_len):
+    """80 short (sequence, KV head) units: CTAs take up to 27 units each in
+    turn, some spanning two CTAs, some empty."""
+    rng = wl.rng_for(8250 + max_len, 3)
+    lens = rng.integers(0, max_len + 1, size=40).tolist()
+    c = Case("fp8", 40, 2, 16, 128, lens, seed=8260 + max_len, factor=16.0)
+    out, lse = run(c)
+    assert int(c.err.item()) == 0
+    assert_close(out, lse, *reference(c))
+
+
 def test_empty_and_single_token():
     c = Case("fp8", 3, 2, 8, 64, [0, 1, 0], seed=8300)
     out, lse = run(c)
@@ -125,7 +138,6 @@ def test_zero_query_closed_form():
     ref_out, ref_lse, amb = reference(c, qs=0.01, ps=ps)
     assert_close(out, lse, ref_out, ref_lse, amb)
     np.testing.assert_allclose(lse, np.log(T), rtol=1e-6)
-    from quantized_kv_cache_21_b200 import workloads as wl
     _, v_hat = oracle.dequantize("fp8", c.okc, c.ovc, 1, 64, wl.physical_slots(c.bt, 0, np.arange(T)),
                                  c.ks, c.vs)
     want = 416.0 * ps * v_hat.astype(np.float64).mean(axis=0)  # E4M3(426.67) = 416

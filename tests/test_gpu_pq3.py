@@ -121,6 +121,18 @@ def test_decode_gqa_ratios(G):
     assert_attention_close(out, lse, *c.reference())
 
 
+@pytest.mark.parametrize("max_len", [16, 100, 700])
+def test_decode_many_units_per_cta(max_len):
+    """80 short (sequence, KV head) units: CTAs take up to 27 units each in
+    turn, some spanning two CTAs, some empty."""
+    rng = wl.rng_for(9560 + max_len, 3)
+    lens = rng.integers(0, max_len + 1, size=40).tolist()
+    c = PQ3Case(40, 2, 16, lens, seed=9570 + max_len, factor=16.0)
+    out, lse = c.decode()
+    assert int(c.err.item()) == 0
+    assert_attention_close(out, lse, *c.reference())
+
+
 def test_decode_long_context_and_splits():
     c = PQ3Case(1, 1, 8, [20000], seed=9540, factor=16.0)
     ref = c.reference()
