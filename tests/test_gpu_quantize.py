@@ -167,6 +167,54 @@ def test_block_table_translation_matches_physical():
     assert np.array_equal(tk, okc) and np.array_equal(tv, ovc)
 
 
+@pytest.mark.parametrize("H,D,T", [(8, 128, 3001), (2, 64, 3001), (32, 128, 1001)])
+def test_large_fp8_write_matches_oracle(H, D, T):
+    """Writes of a thousand and more tokens (8 tokens per block, grid of
+    hundreds of blocks, a ragged last block): logical slots through a block
+    table, skipped tokens and one slot past the last sequence, bit-exact
+    against the oracle; a bad K scale writes no K byte and still writes V."""
+    rng = wl.rng_for(79 + H + D, 0)
+    B = 3
+    mb = -(-T // (16 * B)) + 2
+    nb = B * mb + 1
+    bt = wl.permuted_block_table(rng, B, mb, nb)
+    outl = wl.outlier_pairs(rng, H, D, per_head=1)
+    k = wl.make_tokens(rng, T, H, D, outl, 16.0)
+    v = wl.make_tokens(rng, T, H, D, outl, 16.0)
+    seq = np.arange(T) % B
+    pos = np.arange(T) // B
+    logical = (seq * mb * 16 + pos).astype(np.int64)
+    physical = np.array([wl.physical_slots(bt, sq, [ps])[0] for sq, ps in zip(seq, pos)], np.int64)
+    logical[[5, 1500 % T, T - 1]] = -1
+    physical[[5, 1500 % T, T - 1]] = -1
+    logical[17] = B * mb * 16 + 3  # a sequence past num_seqs: reported, skipped
+    physical[17] = -1
+    ks = oracle.fp8_scale(oracle.absmax_bf16(k[:200]))  # later outliers saturate
+    vs = oracle.fp8_scale(oracle.absmax_bf16(v[:200]))
+    okc, ovc = oracle.new_cache("fp8", nb, H, D, fill=0x5A)
+    oracle.write("fp8", k, v, physical, okc, ovc, ks, vs)
+    cache = kvq.KVCache("fp8", nb, H, D)
+    cache.k.fill_(0x5A)
+    cache.v.fill_(0x5A)
+    err = new_err()
+    kvq.kv_quantize_write("fp8", to_dev_bits(k), to_dev_bits(v), torch.from_numpy(logical).to(DEV),
+                          cache, dev_scalar(ks), dev_scalar(vs), err,
+                          block_table=torch.from_numpy(bt).to(DEV))
+    gk, gv = cache_bytes(cache)
+    assert int(err.item()) == kvq.DERR_SLOT
+    assert np.array_equal(gk, okc) and np.array_equal(gv, ovc)
+    # a bad K scale on a large write: no K byte is written, V still is
+    cache.k.fill_(0x5A)
+    cache.v.fill_(0x5A)
+    e = new_err()
+    kvq.kv_quantize_write("fp8", to_dev_bits(k), to_dev_bits(v), torch.from_numpy(logical).to(DEV),
+                          cache, dev_scalar(float("nan")), dev_scalar(vs), e,
+                          block_table=torch.from_numpy(bt).to(DEV))
+    gk, gv = cache_bytes(cache)
+    assert int(e.item()) == kvq.DERR_SLOT | kvq.DERR_SCALE
+    assert np.all(gk == 0x5A) and np.array_equal(gv, ovc)
+
+
 def test_bad_slots_and_scales_are_reported_not_written():
     rng = wl.rng_for(78, 0)
     H, D, nb = 1, 64, 2
