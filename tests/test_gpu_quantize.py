@@ -38,11 +38,18 @@ def write_both(fmt, k, v, slots, nb, ks, vs, fill=0):
 
 
 @pytest.mark.parametrize("scale", [1.0, 0.125, 3.0517578125e-05, 0.0234375, 1e-12, 0.7,
-                                   33333.0, oracle.scale_from_absmax("fp8", 7.3)])
+                                   33333.0, oracle.scale_from_absmax("fp8", 7.3),
+                                   1.0 / 3.0, 3.0, 7.0, 11.0, 0.3, 3.1415927, 0.0098765, 271.828,
+                                   5.5e-7, 1.7e-10,
+                                   oracle.scale_from_absmax("fp8", 81.25),
+                                   oracle.scale_from_absmax("fp8", 4.6)])
 def test_fp8_every_bf16_input(scale):
     """All 65,280 finite BF16 values through x / s -> E4M3 (s = 1 makes it the
     bare encoder; the other scales move every value across binades; scales
-    that are not powers of two make x / s a true division)."""
+    that are not powers of two make x / s a true division; with s = 3, 7, 11
+    or 0.3 a reciprocal product x * RN(1/s) would encode some inputs
+    differently, e.g. 3.1875 / 3 = 1.0625 is a tie that the product lifts
+    above)."""
     bits = all_finite_bf16()
     H, D = 1, 64
     T = bits.size // D  # 65280 = 1020 * 64
