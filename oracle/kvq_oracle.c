@@ -736,8 +736,14 @@ int orc_decode_attention_fp8qp(const uint16_t* q, const uint8_t* k_cache, const 
  * The dequantised element (fp32): with Y0 = c[i_2j], Y1 = c[i_2j+1],
  *   x_hat_2j = nrm * fmaf(c_j, Y0, s_j * Y1), x_hat_2j+1 = nrm * fmaf(c_j, Y1, -(s_j * Y0)).
  * Layout of a 16-token head page (832 bytes): the 16 norms (fp32), then 16
- * rows of 48 index bytes; index i of a row sits in bits [3i, 3i+3) of the
- * row's little-endian bit string.
+ * rows of 48 index bytes.  A row is two bit planes of its 128 indices, as a
+ * little-endian bit string of 384 bits (the page fixes only the 3 bits an
+ * index; the planes let a reader turn indices into byte-permute selectors
+ * with a few masks):
+ *   low plane, bits 0..255: the low 2 bits of index i = 16w + e (e < 16) at
+ *     bit 32w + 4 (e % 8) + 2 (e / 8);
+ *   high plane, bits 256..383: bit 2 of index i = 32v + e (e < 32) at bit
+ *     256 + 32v + 4 (e % 8) + {2, 3, 0, 1}[e / 8].
  * The per-layer parameter block of a tensor (K or V): 8 codebook values then
  * the 64 (cos, sin) pairs, 136 fp32.
  */
@@ -836,17 +842,35 @@ static void pq3_decode(float nrm, const uint8_t* idx, const float* params, float
   }
 }
 
+/* Bit positions (in the row's 384-bit string) of index i's three bits:
+ * bit k of the index at pq3_bit(i, k). */
+static int pq3_bit(int i, int k) {
+  static const int high_slot[4] = {2, 3, 0, 1};
+  if (k < 2) {
+    const int e = i % 16;
+    return 32 * (i / 16) + 4 * (e % 8) + 2 * (e / 8) + k;
+  }
+  const int e = i % 32;
+  return 256 + 32 * (i / 32) + 4 * (e % 8) + high_slot[e / 8];
+}
+
 static void pq3_pack(const uint8_t* idx, uint8_t* bytes48) {
   for (int b = 0; b < 48; b++) bytes48[b] = 0;
   for (int i = 0; i < ORC_PQ3_D; i++)
     for (int k = 0; k < 3; k++)
-      if ((idx[i] >> k) & 1) bytes48[(3 * i + k) / 8] |= (uint8_t)(1u << ((3 * i + k) % 8));
+      if ((idx[i] >> k) & 1) {
+        const int b = pq3_bit(i, k);
+        bytes48[b / 8] |= (uint8_t)(1u << (b % 8));
+      }
 }
 
 static void pq3_unpack(const uint8_t* bytes48, uint8_t* idx) {
   for (int i = 0; i < ORC_PQ3_D; i++) {
     int v = 0;
-    for (int k = 0; k < 3; k++) v |= ((bytes48[(3 * i + k) / 8] >> ((3 * i + k) % 8)) & 1) << k;
+    for (int k = 0; k < 3; k++) {
+      const int b = pq3_bit(i, k);
+      v |= ((bytes48[b / 8] >> (b % 8)) & 1) << k;
+    }
     idx[i] = (uint8_t)v;
   }
 }

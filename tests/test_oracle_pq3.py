@@ -127,9 +127,11 @@ def test_block_bytes_and_reconstruction_match_the_page():
 
 
 def test_bit_layout_of_a_page():
-    """A 16-token head page: the 16 fp32 norms, then 16 rows of 48 bytes;
-    index i of a row in bits [3i, 3i+3) of the row's little-endian bit
-    string (rebuilt here with numpy's packbits)."""
+    """A 16-token head page: the 16 fp32 norms, then 16 rows of 48 bytes.  A
+    row is 8 little-endian 32-bit words of the indices' low 2 bits (word w:
+    indices 16w + k at bits 4k and 16w + 8 + k at bits 4k + 2, k < 8), then
+    4 words of their high bits (word v: indices 32v + 8j + k at bit
+    4k + (2, 3, 0, 1)[j]); rebuilt here with numpy shifts and sums."""
     pr = params(6)
     rng = wl.rng_for(79, 0)
     x = wl.make_tokens(rng, 1, 1, 128, [(0, 7)], 16.0)
@@ -137,8 +139,13 @@ def test_bit_layout_of_a_page():
     kc, vc = oracle.new_cache("pq3", 1, 1, 128)
     oracle.pq3_write(x, x, np.array([3]), kc, vc, pr, pr)
     assert kc[12:16].view(np.float32)[0] == np.float32(nrm)  # slot 3's norm
-    bits = ((idx[:, None] >> np.arange(3)[None, :]) & 1).astype(np.uint8).reshape(-1)
-    want = np.packbits(bits, bitorder="little")
+    idx = idx.astype(np.uint64)
+    low = (idx & 3).reshape(8, 2, 8)  # [word][half][k]: index 16 w + 8 half + k
+    low_words = (low << (4 * np.arange(8, dtype=np.uint64) + 2 * np.arange(2, dtype=np.uint64)[:, None])).sum(axis=(1, 2))
+    high = (idx >> 2).reshape(4, 4, 8)  # [word][j][k]: index 32 v + 8 j + k
+    slot_of_j = np.array([2, 3, 0, 1], dtype=np.uint64)[:, None]
+    high_words = (high << (4 * np.arange(8, dtype=np.uint64) + slot_of_j)).sum(axis=(1, 2))
+    want = np.concatenate([low_words, high_words]).astype("<u4").view(np.uint8)
     assert want.size == 48
     assert np.array_equal(kc[64 + 3 * 48: 64 + 4 * 48], want)
     # every other byte of the page is untouched
