@@ -80,8 +80,11 @@
  * y_2j = fma(cos_j, u_2j, -(sin_j * u_2j+1)), y_2j+1 = fma(sin_j, u_2j,
  * cos_j * u_2j+1), index = the number of thresholds (c_k + c_k+1) / 2 below
  * y; an all-zero x stores norm 0 and indices 0.
- *   Head page (832 bytes): 16 fp32 norms, then 16 rows of 48 bytes; index i
- *   of a row sits in bits [3i, 3i+3) of the row's little-endian bit string.
+ *   Head page (832 bytes): 16 fp32 norms, then 16 rows of 48 bytes.  A row
+ *   is 12 little-endian 32-bit words in two bit planes: words 0-7 hold the
+ *   low 2 bits of the indices (word w: index 16w + k at bits 4k, 4k+1 and
+ *   index 16w + 8 + k at bits 4k+2, 4k+3, k < 8), words 8-11 their high bits
+ *   (word 8 + v: bit 2 of index 32v + 8j + k at bit 4k + (2, 3, 0, 1)[j]).
  *   The "scale" of a PQ3 tensor (d_k_scale, d_v_scale) is a device array of
  *   136 fp32: the 8 codebook values (f16-representable, ascending; see
  *   kv_pq3_codebook), then the 64 (cos, sin) pairs.

@@ -549,10 +549,14 @@ struct Fmt<2, 128> {
 };
 
 // ---- PQ3 (3-bit planar-rotation codec of 128-element vectors), head_dim 128:
-// a head page is 16 fp32 norms and 16 rows of 48 index bytes (832 B; index i
-// of a row in bits [3i, 3i+3)), fetched whole by bulk copies, K's page then
-// V's.  Indices become exact f16 codebook values by two byte permutes over
-// the codebook's low and high bytes (tl, th), four values at a time.
+// a head page is 16 fp32 norms and 16 rows of 48 index bytes (832 B), fetched
+// whole by bulk copies, K's page then V's.  A row is two bit planes: 8 words
+// of the indices' low 2 bits (word w: index 16w + k at bits 4k, 4k+1 and
+// 16w + 8 + k at bits 4k+2, 4k+3) and 4 words of their high bits (word v:
+// index 32v + 8j + k at bit 4k + (2, 3, 0, 1)[j]).  Two masks and an OR turn
+// a low word and its high bits into 8 byte-permute selectors (one index a
+// nibble); two permutes over the codebook's low and high bytes (tl, th) then
+// give four exact f16 codebook values.
 template <>
 struct Fmt<3, 128> {
   static constexpr bool kBF16 = false;
@@ -576,81 +580,91 @@ struct Fmt<3, 128> {
     bulk_prefetch_l2(page(p.kc, p, h, blk), PAGE);
     bulk_prefetch_l2(page(p.vc, p, h, blk), PAGE);
   }
-  // Raw stage words: K rows gid, gid+8, their norms and the 12 index bytes of
-  // head-dim elements 32tig .. 32tig+31; V rows 2tig, 2tig+1, 2tig+8, 2tig+9,
-  // the 8 aligned bytes holding the indices of elements 16gid .. 16gid+15
-  // (bits [48 gid, 48 gid + 48) of the row), and the V norms of tokens gid and
-  // gid+8 (the token rows of P).
+  // Raw stage words: K rows gid, gid+8 (low words 2tig, 2tig+1 and high word
+  // tig: indices of head-dim elements 32tig .. 32tig+31) and their norms; V
+  // rows 2tig, 2tig+1, 2tig+8, 2tig+9 (low word gid and high word gid / 2:
+  // elements 16gid .. 16gid+15) and the V norms of tokens gid, gid+8 (the
+  // token rows of P).
   struct Raw {
-    uint32_t kw[2][3], vw[4][2];
+    uint2 kl[2];
+    uint32_t kh[2], vl[4], vh[4];
     float nk[2], nv[2];
   };
   __device__ static void load_raw_k(const uint8_t* st, int gid, int tig, Raw& r) {
 #pragma unroll
     for (int rr = 0; rr < 2; ++rr) {
       const int row = gid + 8 * rr;
-      const uint32_t* w = reinterpret_cast<const uint32_t*>(st + 64 + 48 * row + 12 * tig);
-      r.kw[rr][0] = w[0];
-      r.kw[rr][1] = w[1];
-      r.kw[rr][2] = w[2];
+      const uint8_t* rw = st + 64 + 48 * row;
+      r.kl[rr] = *reinterpret_cast<const uint2*>(rw + 8 * tig);
+      r.kh[rr] = *reinterpret_cast<const uint32_t*>(rw + 32 + 4 * tig);
       r.nk[rr] = reinterpret_cast<const float*>(st)[row];
     }
   }
   __device__ static void load_raw_v(const uint8_t* st, int gid, int tig, Raw& r) {
     const uint8_t* sv = st + V_OFF;
-    const int base = (6 * gid) & ~3;
     const int rows[4] = {2 * tig, 2 * tig + 1, 2 * tig + 8, 2 * tig + 9};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const uint32_t* w = reinterpret_cast<const uint32_t*>(sv + 64 + 48 * rows[i] + base);
-      r.vw[i][0] = w[0];
-      r.vw[i][1] = w[1];
+      const uint8_t* rw = sv + 64 + 48 * rows[i];
+      r.vl[i] = *reinterpret_cast<const uint32_t*>(rw + 4 * gid);
+      r.vh[i] = *reinterpret_cast<const uint32_t*>(rw + 32 + 4 * (gid >> 1));
     }
     r.nv[0] = reinterpret_cast<const float*>(sv)[gid];
     r.nv[1] = reinterpret_cast<const float*>(sv)[gid + 8];
   }
-  // f16x2 (c[i0], c[i1]) and (c[i2], c[i3]) of four 3-bit indices.
-  __device__ static void lookup4(uint32_t i0, uint32_t i1, uint32_t i2, uint32_t i3,
-                                 const uint32_t tl[2], const uint32_t th[2], uint32_t& p01,
-                                 uint32_t& p23) {
-    const uint32_t sel = i0 | (i1 << 4) | (i2 << 8) | (i3 << 12);
-    const uint32_t lo = prmt(tl[0], tl[1], sel), hi = prmt(th[0], th[1], sel);
-    p01 = prmt(lo, hi, 0x5140);
-    p23 = prmt(lo, hi, 0x7362);
+  // Selectors of a low word w and its high bits h (bit 4k+2: index k, bit
+  // 4k+3: index 8+k): nibble k of a = index k, nibble k of b = index 8+k.
+  __device__ static void selectors(uint32_t w, uint32_t h, uint32_t& a, uint32_t& b) {
+    a = (w & 0x33333333u) | (h & 0x44444444u);
+    b = ((w >> 2) & 0x33333333u) | ((h >> 1) & 0x44444444u);
   }
-  // A fragments of QK: k-step s takes the 12-bit field at bit 12s of the
-  // thread's 96-bit run (elements 32tig + 4s .. +3).
+  // Bytes [c[n0], c[n1], c[n2], c[n3]] of the selector's low 16 bits, low
+  // bytes in lo and high bytes in hi.
+  __device__ static void lookup(uint32_t sel, const uint32_t tl[2], const uint32_t th[2],
+                                uint32_t& lo, uint32_t& hi) {
+    lo = prmt(tl[0], tl[1], sel);
+    hi = prmt(th[0], th[1], sel);
+  }
+  // A fragments of QK: k-step s takes elements 32tig + 4s .. +3, selector
+  // half s of (a0, b0, a1, b1) in turn.
   __device__ static void conv_k(const Raw& r, uint32_t ka[8][4], const uint32_t tl[2],
                                 const uint32_t th[2]) {
 #pragma unroll
-    for (int s = 0; s < 8; ++s) {
+    for (int rr = 0; rr < 2; ++rr) {
+      uint32_t sel[4];
+      selectors(r.kl[rr].x, r.kh[rr], sel[0], sel[1]);       // elements 0-7, 8-15
+      selectors(r.kl[rr].y, r.kh[rr] << 2, sel[2], sel[3]);  // elements 16-23, 24-31
 #pragma unroll
-      for (int rr = 0; rr < 2; ++rr) {
-        const int b = 12 * s, wi = b >> 5, sh = b & 31;
-        const uint32_t f =
-            (sh + 12 <= 32 ? (r.kw[rr][wi] >> sh) : __funnelshift_r(r.kw[rr][wi], r.kw[rr][wi + 1], sh)) &
-            0xFFFu;
-        lookup4(f & 7u, (f >> 3) & 7u, (f >> 6) & 7u, (f >> 9) & 7u, tl, th, ka[s][rr],
-                ka[s][2 + rr]);
+      for (int s = 0; s < 8; ++s) {
+        uint32_t lo, hi;
+        lookup((s & 1) ? sel[s >> 1] >> 16 : sel[s >> 1], tl, th, lo, hi);
+        ka[s][rr] = prmt(lo, hi, 0x5140);      // elements 4s, 4s+1
+        ka[s][2 + rr] = prmt(lo, hi, 0x7362);  // elements 4s+2, 4s+3
       }
     }
   }
   // A fragments of PV: m-tile jj takes head-dim elements 16gid + 2jj, +1 of
   // tokens 2tig, 2tig+1 (va[jj][0], [1]) and 2tig+8, 2tig+9 (va[jj][2], [3]).
+  // Selector byte jj & 3 of a row holds both elements' indices; one permute
+  // puts two token rows' bytes side by side.
   __device__ static void conv_v(const Raw& r, uint32_t va[8][4], const uint32_t tl[2],
                                 const uint32_t th[2], int gid) {
-    const int sh0 = ((6 * gid) & 3) * 8;  // the run starts 0 or 16 bits into the words
-    uint64_t run[4];
+    const int hs = 2 * (gid & 1);  // odd gid: the high word's upper 16 indices
+    uint32_t sa[4], sb[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
-      run[i] = ((static_cast<uint64_t>(r.vw[i][1]) << 32) | r.vw[i][0]) >> sh0;
+    for (int i = 0; i < 4; ++i) selectors(r.vl[i], r.vh[i] << hs, sa[i], sb[i]);
 #pragma unroll
     for (int jj = 0; jj < 8; ++jj) {
-      uint32_t f[4];
+      const uint32_t pick = (jj & 3) | ((4 + (jj & 3)) << 4);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) f[i] = static_cast<uint32_t>(run[i] >> (6 * jj)) & 63u;
-      lookup4(f[0] & 7u, f[1] & 7u, f[0] >> 3, f[1] >> 3, tl, th, va[jj][0], va[jj][1]);
-      lookup4(f[2] & 7u, f[3] & 7u, f[2] >> 3, f[3] >> 3, tl, th, va[jj][2], va[jj][3]);
+      for (int pr = 0; pr < 2; ++pr) {  // token rows (2tig, 2tig+1), then (2tig+8, 2tig+9)
+        const uint32_t x = jj < 4 ? sa[2 * pr] : sb[2 * pr];
+        const uint32_t y = jj < 4 ? sa[2 * pr + 1] : sb[2 * pr + 1];
+        uint32_t lo, hi;
+        lookup(prmt(x, y, pick), tl, th, lo, hi);
+        va[jj][2 * pr] = prmt(lo, hi, 0x6240);      // element 2jj of both rows
+        va[jj][2 * pr + 1] = prmt(lo, hi, 0x7351);  // element 2jj+1
+      }
     }
   }
 };
