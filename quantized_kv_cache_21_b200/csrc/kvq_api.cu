@@ -120,6 +120,14 @@ kvq_status make_plan(int32_t fmt, int32_t B, int32_t Hq, int32_t Hkv, int32_t D,
   } else {
     ctas = V / (2 * cfg.warps);  // at least two pages per consumer warp
     if (ctas > sms) ctas = sms;
+    // With few units, a whole number of CTAs per unit (if that leaves at
+    // most a tenth of the CTAs out) keeps every CTA inside one unit: a CTA
+    // whose range held two units would scan them in turn, with a merge
+    // between, and end last.
+    if (ctas > units && ctas % units != 0) {
+      const int64_t whole = ctas / units * units;
+      if (whole * 10 >= ctas * 9) ctas = whole;
+    }
   }
   if (V > 0 && ctas > V) ctas = V;
   if (ctas > 4096) ctas = 4096;
