@@ -120,13 +120,15 @@ kvq_status make_plan(int32_t fmt, int32_t B, int32_t Hq, int32_t Hkv, int32_t D,
   } else {
     ctas = V / (2 * cfg.warps);  // at least two pages per consumer warp
     if (ctas > sms) ctas = sms;
-    // With few units, a whole number of CTAs per unit (if that leaves at
-    // most a tenth of the CTAs out) keeps every CTA inside one unit: a CTA
-    // whose range held two units would scan them in turn, with a merge
-    // between, and end last.
+    // With fewer units than CTAs, a whole number of CTAs per unit keeps
+    // every CTA inside one unit: a CTA whose range held two units would scan
+    // them in turn, with a merge between (~6-8 us), and end last.  Taken if
+    // it leaves at most a tenth of the CTAs out, or if each CTA then scans at
+    // most ~96 more pages (about what that merge costs at 12 pages a us).
     if (ctas > units && ctas % units != 0) {
       const int64_t whole = ctas / units * units;
-      if (whole * 10 >= ctas * 9) ctas = whole;
+      const int64_t extra = V / whole - V / ctas;
+      if (whole * 10 >= ctas * 9 || extra <= 96) ctas = whole;
     }
   }
   if (V > 0 && ctas > V) ctas = V;
