@@ -906,7 +906,6 @@ __global__ void __launch_bounds__(Shape<FMT, D>::NW * 32, 1)
       scale_ok = ks > 0.f && vs > 0.f && ks < kInf && vs < kInf;
     else
       scale_ok = ks >= 0.f && vs >= 0.f && ks < kInf && vs < kInf;
-    if (!scale_ok && c == 0 && tid == 0) set_err(p.d_err, kErrScale);
   } else if constexpr (FMT == 3) {
 #pragma unroll
     for (int kv = 0; kv < 2; ++kv) {
@@ -926,7 +925,6 @@ __global__ void __launch_bounds__(Shape<FMT, D>::NW * 32, 1)
       th[0] = prmt(w01, w23, 0x7531);  // high bytes
       th[1] = prmt(w45, w67, 0x7531);
     }
-    if (!scale_ok && c == 0 && tid == 0) set_err(p.d_err, kErrScale);
   }
   // FP8 attention: the E4M3 scales of q and P (both > 0 and finite).  The
   // output takes prob_scale, and the 2^kPLog2 that l carries (see pv_page).
@@ -934,11 +932,7 @@ __global__ void __launch_bounds__(Shape<FMT, D>::NW * 32, 1)
   if constexpr (QP) {
     qs = __ldg(p.q_scale);
     const float ps = __ldg(p.prob_scale);
-    const bool ok = qs > 0.f && qs < kInf && ps > 0.f && ps < kInf;
-    if (!ok) {
-      if (scale_ok && c == 0 && tid == 0) set_err(p.d_err, kErrScale);
-      scale_ok = false;
-    }
+    scale_ok = scale_ok && qs > 0.f && qs < kInf && ps > 0.f && ps < kInf;
     inv_ps = __fdiv_rn(1.f, ps);
     vs_out = vs * ps * 4096.f;  // 2^kPLog2
   }
@@ -977,19 +971,27 @@ __global__ void __launch_bounds__(Shape<FMT, D>::NW * 32, 1)
     else
       F::conv_v(raw, va);
   };
-  auto load_q = [&](int u) {
+  // q of unit u in two steps: fetch_q issues the loads of the thread's
+  // head-dim runs (zero for padded heads), conv_q builds the fragments, so
+  // the first unit's loads overlap the other prologue loads.
+  using QRaw = uint4[D / 32];
+  auto fetch_q = [&](int u, QRaw& w) {
     const int grp = u % p.n_groups, h = (u / p.n_groups) % p.Hkv, b = u / (p.n_groups * p.Hkv);
     const int qi = grp * 8 + gid;
     const bool hv = qi < p.G;
     const uint16_t* qrow = p.q + (static_cast<size_t>(b) * p.Hq + h * p.G + (hv ? qi : 0)) * D;
+#pragma unroll
+    for (int s = 0; s < D / 32; ++s)
+      w[s] = hv ? __ldg(reinterpret_cast<const uint4*>(qrow + F::k_elem(tig, 8 * s)))
+                : make_uint4(0u, 0u, 0u, 0u);
+  };
+  auto conv_q = [&](const QRaw& w) {
     if constexpr (QP) {
       // q_hat = E4M3(q / q_scale): IEEE fp32 division, round to nearest even,
       // saturating (the rounding of the cache write)
 #pragma unroll
       for (int s = 0; s < D / 32; ++s) {
-        const uint4 w = hv ? __ldg(reinterpret_cast<const uint4*>(qrow + F::k_elem(tig, 8 * s)))
-                           : make_uint4(0u, 0u, 0u, 0u);
-        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+        const uint32_t ws[4] = {w[s].x, w[s].y, w[s].z, w[s].w};
         uint32_t e[4];
 #pragma unroll
         for (int x = 0; x < 4; ++x)
@@ -1001,9 +1003,7 @@ __global__ void __launch_bounds__(Shape<FMT, D>::NW * 32, 1)
       const float* rot = p.k_scale + 8;
 #pragma unroll
       for (int i = 0; i < D / 4; i += 8) {
-        const uint4 w = hv ? __ldg(reinterpret_cast<const uint4*>(qrow + F::k_elem(tig, i)))
-                           : make_uint4(0u, 0u, 0u, 0u);
-        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+        const uint32_t ws[4] = {w[i / 8].x, w[i / 8].y, w[i / 8].z, w[i / 8].w};
 #pragma unroll
         for (int x = 0; x < 4; ++x) {  // the pair of head-dim elements 2j, 2j+1
           const int j = F::k_elem(tig, i) / 2 + x;
@@ -1020,9 +1020,7 @@ __global__ void __launch_bounds__(Shape<FMT, D>::NW * 32, 1)
     } else {
 #pragma unroll
       for (int i = 0; i < D / 4; i += 8) {
-        const uint4 w = hv ? __ldg(reinterpret_cast<const uint4*>(qrow + F::k_elem(tig, i)))
-                           : make_uint4(0u, 0u, 0u, 0u);
-        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+        const uint32_t ws[4] = {w[i / 8].x, w[i / 8].y, w[i / 8].z, w[i / 8].w};
 #pragma unroll
         for (int x = 0; x < 4; ++x) {
           uint32_t v = ws[x];
@@ -1032,7 +1030,13 @@ __global__ void __launch_bounds__(Shape<FMT, D>::NW * 32, 1)
       }
     }
   };
-  load_q(u0);  // in flight while the unit table is built
+  auto load_q = [&](int u) {
+    QRaw w;
+    fetch_q(u, w);
+    conv_q(w);
+  };
+  QRaw q0raw;
+  fetch_q(u0, q0raw);  // in flight while the unit table is built
 
   // Block ids of this warp's first 64 local items, loaded now on the guess
   // that they lie in unit u0 (they do unless its segment is shorter), so they
@@ -1079,6 +1083,10 @@ __global__ void __launch_bounds__(Shape<FMT, D>::NW * 32, 1)
       tab.total = run;
     }
   }
+  // The scales' check is reported here, after the table, so that no thread
+  // waits on the scale loads before the other prologue loads are issued.
+  if (c == 0 && tid == 0 && !scale_ok) set_err(p.d_err, kErrScale);
+  conv_q(q0raw);
   // Ask L2 for the pages of this warp's first stages (the guessed block ids)
   // while the unit table is built; a wrong guess only costs a prefetch.
   if (p.window <= 0 && lane < NSW && spec0 >= 0 && spec0 < p.num_blocks)
