@@ -1087,9 +1087,11 @@ __global__ void __launch_bounds__(Shape<FMT, D>::NW * 32, 1)
   // waits on the scale loads before the other prologue loads are issued.
   if (c == 0 && tid == 0 && !scale_ok) set_err(p.d_err, kErrScale);
   conv_q(q0raw);
-  // Ask L2 for the pages of this warp's first stages (the guessed block ids)
-  // while the unit table is built; a wrong guess only costs a prefetch.
-  if (p.window <= 0 && lane < NSW && spec0 >= 0 && spec0 < p.num_blocks)
+  // Ask L2 for the page of this warp's first stage (the guessed block id)
+  // while the unit table is built; a wrong guess only costs a prefetch.  Only
+  // the first: prefetching the pages of all NSW stages measured slower on the
+  // head_dim-64 decodes (1 x 65,536 tokens: NVFP4 30.7 against 28.7 us).
+  if (p.window <= 0 && lane == 0 && spec0 >= 0 && spec0 < p.num_blocks)
     F::prefetch(&mk, &mv, (u0 / p.n_groups) % p.Hkv, spec0, p);
   if (lane < NSW) mbar_init(&bars[lane], 1);  // each warp its own stages
   mbar_init_fence();
