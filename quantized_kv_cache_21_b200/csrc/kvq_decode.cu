@@ -102,6 +102,7 @@ struct Fmt<1, 128> {
     uint4 k[4], v[4];
   };
   static constexpr bool kLateV = false;
+  static constexpr bool kStream = false;
   __device__ static void load_raw_k(const uint8_t* st, int gid, int tig, Raw& r) {
 #pragma unroll
     for (int rr = 0; rr < 2; ++rr) {
@@ -164,6 +165,7 @@ struct Fmt<1, 64> {
     uint2 v[4];
   };
   static constexpr bool kLateV = false;
+  static constexpr bool kStream = false;
   __device__ static void load_raw_k(const uint8_t* st, int gid, int tig, Raw& r) {
 #pragma unroll
     for (int rr = 0; rr < 2; ++rr) r.k[rr] = lds128(st + swz64(gid + 8 * rr, 16 * tig));
@@ -220,6 +222,7 @@ struct Fmt<0, 64> {
     uint4 k[4], v[4];
   };
   static constexpr bool kLateV = false;
+  static constexpr bool kStream = false;
   __device__ static void load_raw_k(const uint8_t* st, int gid, int tig, Raw& r) {
 #pragma unroll
     for (int rr = 0; rr < 2; ++rr) {
@@ -294,6 +297,7 @@ struct Fmt<0, 128> {
   // 64 raw registers would not fit beside the accumulators: K is read and
   // used first, V read after the QK product (kLateV), then the stage refilled.
   static constexpr bool kLateV = true;
+  static constexpr bool kStream = false;
   __device__ static void load_raw_k(const uint8_t* st, int gid, int tig, Raw& r) {
 #pragma unroll
     for (int hf = 0; hf < 2; ++hf) {
@@ -391,6 +395,7 @@ struct Fmt<2, 64> {
     uint32_t v[4], ks[2], vs[4];
   };
   static constexpr bool kLateV = false;
+  static constexpr bool kStream = false;
   __device__ static void load_raw_k(const uint8_t* st, int gid, int tig, Raw& r) {
 #pragma unroll
     for (int rr = 0; rr < 2; ++rr) {
@@ -479,6 +484,10 @@ struct Fmt<2, 128> {
     uint32_t ks[2], vs[4];
   };
   static constexpr bool kLateV = false;
+  // K decoded per pair of k-steps right at its MMAs and V four m-tiles at a
+  // time after the softmax, so no whole page of fragments is live at once
+  // (154 registers instead of 164; the 4 x 126,976-token decode 180 -> 174 us)
+  static constexpr bool kStream = true;
   __device__ static void load_raw_k(const uint8_t* st, int gid, int tig, Raw& r) {
 #pragma unroll
     for (int rr = 0; rr < 2; ++rr) {
@@ -518,6 +527,48 @@ struct Fmt<2, 128> {
         ka[s][rr] = hmul2(f[2 * s], sc);
         ka[s][2 + rr] = hmul2(f[2 * s + 1], sc);
       }
+    }
+  }
+  // k-steps 2w and 2w+1 only: code word w of both rows (blocks 2tig for
+  // w < 2, 2tig+1 after), the same values conv_k puts in ka[2w], ka[2w+1]
+  __device__ static void conv_k_pair(const Raw& r, int w, uint32_t a0[4], uint32_t a1[4]) {
+#pragma unroll
+    for (int rr = 0; rr < 2; ++rr) {
+      uint32_t s01, unused;
+      e4m3x4_to_f16x2x2(r.ks[rr], s01, unused);
+      const uint32_t sc = w < 2 ? prmt(s01, s01, 0x1010) : prmt(s01, s01, 0x3232);
+      const uint4 c = r.k[rr];
+      const uint32_t word = w == 0 ? c.x : w == 1 ? c.y : w == 2 ? c.z : c.w;
+      uint32_t f[4];
+      e2m1x8_to_f16x2x4(word, f);
+      a0[rr] = hmul2(f[0], sc);
+      a0[2 + rr] = hmul2(f[1], sc);
+      a1[rr] = hmul2(f[2], sc);
+      a1[2 + rr] = hmul2(f[3], sc);
+    }
+  }
+  // m-tiles 4wi .. 4wi+3 only: the values conv_v puts in va[4wi .. 4wi+3]
+  __device__ static void conv_v_half(const Raw& r, int wi, uint32_t va[4][4]) {
+    const uint32_t sxy = scale_pair(r.vs[0], r.vs[1]);
+    const uint32_t szw = scale_pair(r.vs[2], r.vs[3]);
+    const uint32_t x = wi ? r.v[0].y : r.v[0].x, y = wi ? r.v[1].y : r.v[1].x;
+    const uint32_t z = wi ? r.v[2].y : r.v[2].x, w = wi ? r.v[3].y : r.v[3].x;
+    uint32_t lo, hi, L[4], H[4];
+    nib_interleave(x, y, lo, hi);
+    e2m1x8_to_f16x2x4(lo, L);
+    e2m1x8_to_f16x2x4(hi, H);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      va[j][0] = hmul2(L[j], sxy);
+      va[j][1] = hmul2(H[j], sxy);
+    }
+    nib_interleave(z, w, lo, hi);
+    e2m1x8_to_f16x2x4(lo, L);
+    e2m1x8_to_f16x2x4(hi, H);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      va[j][2] = hmul2(L[j], szw);
+      va[j][3] = hmul2(H[j], szw);
     }
   }
   __device__ static void conv_v(const Raw& r, uint32_t va[8][4]) {
@@ -562,6 +613,7 @@ struct Fmt<3, 128> {
   static constexpr bool kBF16 = false;
   static constexpr int STAGE = 1664, TX = 1664, V_OFF = 832, PAGE = 832;
   static constexpr bool kLateV = false;
+  static constexpr bool kStream = false;
   __device__ static int k_elem(int tig, int i) { return 32 * tig + i; }
   __device__ static int v_elem(int gid, int i) { return 16 * gid + i; }
   __device__ static const uint8_t* page(const uint8_t* base, const DecodeParams& p, int h,
@@ -1508,6 +1560,16 @@ __global__ void __launch_bounds__(Shape<FMT, D>::NW * 32, 1)
         float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
         // ---- S^T = K Q^T on tensor cores (two accumulator chains)
         auto qk = [&]() {
+          if constexpr (F::kStream) {
+  #pragma unroll
+            for (int w = 0; w < KS / 2; ++w) {
+              uint32_t a0[4], a1[4];
+              F::conv_k_pair(raw, w, a0, a1);
+              mma16816<F::kBF16>(sa, a0, qb[2 * w][0], qb[2 * w][1]);
+              mma16816<F::kBF16>(sb, a1, qb[2 * w + 1][0], qb[2 * w + 1][1]);
+            }
+            return;
+          }
           conv_k_any(raw, ka);
   #pragma unroll
           for (int s = 0; s < KS; ++s) {
@@ -1539,7 +1601,7 @@ __global__ void __launch_bounds__(Shape<FMT, D>::NW * 32, 1)
         }
         if (!valid) continue;
         if constexpr (!F::kLateV) qk();
-        conv_v_any(raw, va);
+        if constexpr (!F::kStream) conv_v_any(raw, va);
 
         // raw scores r = q . k_code (the scale c_log2 is applied below)
         float r0 = sa[0] + sb[0], r1 = sa[1] + sb[1], r2 = sa[2] + sb[2], r3 = sa[3] + sb[3];
@@ -1549,6 +1611,7 @@ __global__ void __launch_bounds__(Shape<FMT, D>::NW * 32, 1)
           r2 *= raw.nk[1];
           r3 *= raw.nk[1];
         }
+        uint32_t vm01 = 0xFFFFFFFFu, vm23 = 0xFFFFFFFFu;  // V token masks of a partial page
         if (k == k_end - 1 && n_last < kPage) {  // last, partial page: mask tokens past the length
           const int n_valid = n_last;
           if (gid >= n_valid) r0 = r1 = -kInf;
@@ -1561,12 +1624,16 @@ __global__ void __launch_bounds__(Shape<FMT, D>::NW * 32, 1)
                                (2 * tig + 1 < n_valid ? 0xFFFF0000u : 0u);
           const uint32_t m23 = (2 * tig + 8 < n_valid ? 0x0000FFFFu : 0u) |
                                (2 * tig + 9 < n_valid ? 0xFFFF0000u : 0u);
+          vm01 = m01;
+          vm23 = m23;
+          if constexpr (!F::kStream) {
   #pragma unroll
-          for (int jj = 0; jj < MT; ++jj) {  // unwritten slots may hold NaN codes
-            va[jj][0] &= m01;
-            va[jj][1] &= m01;
-            va[jj][2] &= m23;
-            va[jj][3] &= m23;
+            for (int jj = 0; jj < MT; ++jj) {  // unwritten slots may hold NaN codes
+              va[jj][0] &= m01;
+              va[jj][1] &= m01;
+              va[jj][2] &= m23;
+              va[jj][3] &= m23;
+            }
           }
         }
         if (n_skip > 0 && ps == 0 && k == k_base) {  // window's first page: tokens before it
@@ -1663,10 +1730,33 @@ __global__ void __launch_bounds__(Shape<FMT, D>::NW * 32, 1)
         const uint32_t bl0 = movmatrix_t(x0l), bl1 = movmatrix_t(x1l);
 
         // ---- O^T += V^T P^T
+        if constexpr (F::kStream) {  // V decoded four m-tiles at a time
+          const bool part = k == k_end - 1 && n_last < kPage;
   #pragma unroll
-        for (int jj = 0; jj < MT; ++jj) {
-          mma16816<F::kBF16>(o[jj], va[jj], bh0, bh1);
-          mma16816<F::kBF16>(o[jj], va[jj], bl0, bl1);
+          for (int wi = 0; wi < MT / 4; ++wi) {
+            uint32_t v4[4][4];
+            F::conv_v_half(raw, wi, v4);
+            if (part) {
+  #pragma unroll
+              for (int x = 0; x < 4; ++x) {  // unwritten slots may hold NaN codes
+                v4[x][0] &= vm01;
+                v4[x][1] &= vm01;
+                v4[x][2] &= vm23;
+                v4[x][3] &= vm23;
+              }
+            }
+  #pragma unroll
+            for (int x = 0; x < 4; ++x) {
+              mma16816<F::kBF16>(o[4 * wi + x], v4[x], bh0, bh1);
+              mma16816<F::kBF16>(o[4 * wi + x], v4[x], bl0, bl1);
+            }
+          }
+        } else {
+  #pragma unroll
+          for (int jj = 0; jj < MT; ++jj) {
+            mma16816<F::kBF16>(o[jj], va[jj], bh0, bh1);
+            mma16816<F::kBF16>(o[jj], va[jj], bl0, bl1);
+          }
         }
       }
     }
