@@ -13,7 +13,9 @@
 //
 // Design (one launch per decode step):
 //   * Work = the virtual page space units x pmax, where a unit is (sequence,
-//     KV head, group of <= 8 query heads) and pmax = ceil(max_seq_len / 16).
+//     KV head, group of <= 8 query heads) and pmax = ceil(max_seq_len / 16)
+//     (plus some empty pages at each unit's end when units straddle CTAs, so
+//     a CTA whose range holds a unit boundary scans fewer pages).
 //     It is cut evenly over persistent CTAs (one per SM), so every SM streams
 //     the same number of pages whatever the batch shape (stream-K style); a
 //     CTA walks its range unit by unit ("segments").
@@ -1093,7 +1095,7 @@ __global__ void __launch_bounds__(Shape<FMT, D>::NW * 32, 1)
   // Block ids of this warp's first 64 local items, loaded now on the guess
   // that they lie in unit u0 (they do unless its segment is shorter), so they
   // share one memory round trip with q, the scales and seq_lens instead of
-  // waiting for the unit table.  Clamped to pmax - 1 <= max_blocks - 1, the
+  // waiting for the unit table.  Clamped to max_blocks - 1, the
   // loads stay in the table row; a wrong guess is discarded below.
   const int g0 = warp + lane * NW, g1 = warp + (32 + lane) * NW;
   int spec0, spec1;
@@ -1101,8 +1103,8 @@ __global__ void __launch_bounds__(Shape<FMT, D>::NW * 32, 1)
     const int32_t* bt0 = p.block_table +
                          static_cast<size_t>(u0 / (p.n_groups * p.Hkv)) * p.max_blocks;
     const int ps0 = ps_of(p, u0, vbeg);
-    spec0 = __ldg(bt0 + min(ps0 + g0, p.pmax - 1));
-    spec1 = __ldg(bt0 + min(ps0 + g1, p.pmax - 1));
+    spec0 = __ldg(bt0 + min(ps0 + g0, p.max_blocks - 1));
+    spec1 = __ldg(bt0 + min(ps0 + g1, p.max_blocks - 1));
   }
 
   // ---- unit table: lane i of warp 0 looks at unit u0 + i (32 at a time)
@@ -1935,6 +1937,9 @@ void config_t(DecodeConfig* c) {
   c->stage_bytes = Fmt<FMT, D>::STAGE;
   c->smem_bytes = smem_bytes<FMT, D>();
   c->part_floats = Shape<FMT, D>::WPART;
+  // measured on the 4 x 126,976 and 8 x 65,536-token decodes (optimum ~96-128
+  // pages; PQ3 pages take about three times as long as FP8 pages)
+  c->merge_pages = FMT == 3 ? 64 : 128;
 }
 
 }  // namespace

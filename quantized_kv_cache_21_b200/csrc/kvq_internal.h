@@ -30,18 +30,21 @@ struct DecodeParams {
   int max_blocks;
   int B, Hq, Hkv, G, n_groups;
   int units;                  // B * Hkv * n_groups (sequence, KV head, group of 8 q heads)
-  int pmax;                   // pages per unit in the work partition: ceil(max_seq_len / 16)
+  int pmax;                   // pages per unit in the work partition: ceil(max_seq_len / 16),
+                              // plus merge_pages of empty padding when units straddle CTAs
   int max_seq_len;
   int window;                 // > 0: attend to each sequence's last `window` tokens only
   float sm_scale;
 };
 
 struct DecodeConfig {
-  int warps;        // consumer warps per CTA (plus one producer warp)
+  int warps;        // warps per CTA
   int stages;       // shared-memory ring stages per CTA
   int stage_bytes;  // bytes per stage
   size_t smem_bytes;
   int part_floats;  // floats of one (m, l, o) partial for 8 heads
+  int merge_pages;  // pages a CTA scans in about the time a unit boundary inside
+                    // its range costs it (the segment merge, the next unit's start)
 };
 
 // Per-(format, head_dim) kernel configuration; false if unsupported.
