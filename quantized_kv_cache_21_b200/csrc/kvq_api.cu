@@ -122,13 +122,29 @@ kvq_status make_plan(int32_t fmt, int32_t B, int32_t Hq, int32_t Hkv, int32_t D,
     if (ctas > sms) ctas = sms;
     // With fewer units than CTAs, a whole number of CTAs per unit keeps
     // every CTA inside one unit: a CTA whose range held two units would scan
-    // them in turn, with a merge between (~6-8 us), and end last.  Taken if
-    // it leaves at most a tenth of the CTAs out, or if each CTA then scans at
-    // most ~96 more pages (about what that merge costs at 12 pages a us).
+    // them in turn, with a merge between (~8-10 us), and end last.  The other
+    // way is to keep all CTAs and pad each unit's share with merge_pages
+    // empty pages (below).
     if (ctas > units && ctas % units != 0) {
       const int64_t whole = ctas / units * units;
-      const int64_t extra = V / whole - V / ctas;
-      if (whole * 10 >= ctas * 9 || extra <= 96) ctas = whole;
+      bool take_whole;
+      if (fmt == KVQ_FMT_BF16) {
+        // BF16 pages stream at the HBM rate whatever the CTA count: whole
+        // CTAs if that leaves out at most a tenth of them or costs each at
+        // most ~96 more pages (4 x 32,768 tokens: 90.2 us whole, 92.2 padded)
+        take_whole = whole * 10 >= ctas * 9 || V / whole - V / ctas <= 96;
+      } else {
+        // the quantized page loops are bound by instruction issue, so every
+        // SM counts: whole CTAs unless the padded split gives each CTA at
+        // least 5% fewer pages.  4 x 32,768 tokens on 148 SMs pads (512
+        // against 471 pages a CTA; FP8 55.4 -> 54.0 us, NVFP4 59.5 -> 56.3);
+        // 4 x 16,384 (256 against 249; 34.8 whole, 36.9 padded) and 8 units
+        // of 65,536 tokens (228 against 228) stay whole.
+        const int64_t per_whole = (V + whole - 1) / whole;
+        const int64_t per_pad = (V + units * cfg.merge_pages + ctas - 1) / ctas;
+        take_whole = per_pad * 105 >= per_whole * 100;
+      }
+      if (take_whole) ctas = whole;
     }
   }
   if (V > 0 && ctas > V) ctas = V;
@@ -139,7 +155,7 @@ kvq_status make_plan(int32_t fmt, int32_t B, int32_t Hq, int32_t Hkv, int32_t D,
   // there for the first unit's merge and starts the next unit.  Each unit's
   // share of the partition gets merge_pages empty pages at its end, so such
   // a CTA scans about that many fewer pages and ends with the others (the
-  // 4 x 126,976-token FP8 decode 170 -> 166 us).  The padding holds no work.
+  // 4 x 126,976-token FP8 decode 167.9 -> 163.8 us).  The padding holds no work.
   if (V > 0 && num_splits == 0 && ctas > units && ctas % units != 0) pl->pmax += cfg.merge_pages;
   // A unit that straddles CTAs is finished from per-CTA partials (one slot
   // per (unit, CTA) pair) with an arrival counter per unit.
