@@ -107,7 +107,7 @@ def measured_tensor_peak():
 def source_digest() -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "quantized_kv_cache_21_b200", "csrc")
-    for name in ("kvq_decode.cu", "kvq_device.cuh"):
+    for name in ("kvq_decode.cu", "kvq_device.cuh", "kvq_api.cu"):  # kernel and its work plan
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
